@@ -1,0 +1,484 @@
+#!/usr/bin/env python
+"""Benchmark of the QLoRA hot path on B200: NF4 + DQ quantize, standalone dequant, fused
+QLoRA linear forward + backward.
+
+One step = the whole path over one batch of synthetic input for the seven linears of a
+LLaMA-13B decoder block (q, k, v, o 5120x5120; gate, up 13824x5120; down 5120x13824), 8192
+tokens per GPU, LoRA r = 64, alpha = 16: for each linear, quantize its bf16 weight (absmax,
+nearest NF4 level, packing, double quantization), dequantize it to bf16 (the standalone HBM
+stream), then the fused forward and the backward (dX, dA, dB).  With N > 1 GPUs each rank
+runs its own 8192-token batch (data parallel, weak scaling) and the adapter gradients are
+summed across ranks with NCCL after each backward.
+
+value = algorithmic fwd+bwd flops of all ranks (4MNK + 6MKr + 6MNr per linear) / step time
+(max over ranks), so quantize and dequant time count against it.  Per-row rates, the
+roofline of the dominant kernel (timed live with CUDA events around its launches), the CPU
+oracle baseline, an end-to-end run through host buffers and the SM clocks seen during the
+timed region are reported on the same JSON line.
+
+--impl reference times the CPU oracle (oracle/) on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "QLoRA linear fwd+bwd TFLOP/s and NF4 dequant GB/s, % of B200 roofline"
+WORKLOAD = "llama13b_block_8192tok"
+R = 64
+ALPHA = 16.0
+M_TOKENS = 8192
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# Algorithmic bytes per weight: quantize reads bf16 (2 B) and writes codes (0.5 B), scale
+# codes (1/64 B) and group constants (4/(64*256) B); dequant reads the latter and writes bf16.
+CODEC_BYTES_PER_WEIGHT = 2.0 + 0.5 + 1.0 / 64 + 4.0 / (64 * 256)
+
+
+def linears():
+    import synth
+    return synth.LLAMA13B
+
+
+def linear_flops(M, N, K, r):
+    return 4 * M * N * K + 6 * M * K * r + 6 * M * N * r
+
+
+def step_flops(M=M_TOKENS, r=R):
+    return sum(linear_flops(M, l.N, l.K, r) for l in linears())
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------------------------------
+# clocks during the timed region
+# ------------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        with open(self.path) as f:
+            for line in f:
+                p = [x.strip() for x in line.split(",")]
+                if len(p) < 9:
+                    continue
+                try:
+                    sm.append(float(p[1]))
+                    smax.append(float(p[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, p[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------------------
+# our arm
+# ------------------------------------------------------------------------------------------
+class LinearBufs:
+    """Device buffers of one linear, preallocated so the timed region allocates nothing."""
+
+    def __init__(self, lin, M, r, seed, dev):
+        import torch
+        import synth
+        import bit_nf4_quantized_dq_b200 as q
+        self.N, self.K, self.M, self.r = lin.N, lin.K, M, r
+        self.s = ALPHA / r
+        self.W = synth.normal_bf16((lin.N, lin.K), 0.02, seed, device=dev)
+        inp = synth.linear_inputs(M, lin.N, lin.K, r, seed, device=dev)
+        self.x, self.A, self.B, self.dY = inp["x"], inp["A"], inp["B"], inp["dY"]
+        numel = lin.N * lin.K
+        nb = (numel + 63) // 64
+        ng = (nb + 255) // 256
+        u8, f32, bf = torch.uint8, torch.float32, torch.bfloat16
+        self.Q = q.NF4Tensor(torch.empty(32 * nb, dtype=u8, device=dev), torch.empty(nb, dtype=u8, device=dev),
+                             torch.empty(ng, dtype=f32, device=dev), torch.empty(1, dtype=f32, device=dev),
+                             (lin.N, lin.K))
+        L = q.lib()
+        self.ws_q = torch.empty(L.nf4_quantize_workspace_bytes(numel), dtype=u8, device=dev)
+        self.ws_f = torch.empty(max(256, L.qlora_linear_fwd_workspace_bytes(M, lin.K, lin.N, r)), dtype=u8,
+                                device=dev)
+        self.ws_b = torch.empty(max(256, L.qlora_linear_bwd_workspace_bytes(M, lin.K, lin.N, r)), dtype=u8,
+                                device=dev)
+        self.y = torch.empty((M, lin.N), dtype=bf, device=dev)
+        self.t = torch.empty((M, r), dtype=f32, device=dev)
+        self.dX = torch.empty((M, lin.K), dtype=bf, device=dev)
+        self.dA = torch.empty((r, lin.K), dtype=bf, device=dev)
+        self.dB = torch.empty((lin.N, r), dtype=bf, device=dev)
+        self.plan = q.linear_plan(M, lin.K, lin.N, r)
+
+
+def _p(t):
+    import ctypes
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def run_linear(L, b: LinearBufs, wdq, stream, ev=None):
+    """quantize -> dequant -> forward -> backward of one linear through the C ABI."""
+    import ctypes
+    import bit_nf4_quantized_dq_b200 as q
+    st = ctypes.c_void_p(stream)
+
+    def chk(rc, what):
+        if rc != 0:
+            raise RuntimeError(f"{what}: {rc} {L.qnf4_last_error().decode()}")
+
+    numel = b.N * b.K
+    if ev:
+        ev["q0"].record()
+    chk(L.nf4_quantize_dq(_p(b.W), numel, _p(b.Q.codes), _p(b.Q.scale_codes), _p(b.Q.c2), _p(b.Q.mean),
+                          _p(b.ws_q), b.ws_q.numel(), st), "quantize")
+    if ev:
+        ev["q1"].record()
+    chk(L.nf4_dequant(_p(b.Q.codes), _p(b.Q.scale_codes), _p(b.Q.c2), _p(b.Q.mean), numel, _p(wdq), st),
+        "dequant")
+    if ev:
+        ev["d1"].record()
+        q.set_timing_events(ev["fwd"])
+    chk(L.qlora_linear_fwd(_p(b.x), b.M, b.K, b.N, _p(b.Q.codes), _p(b.Q.scale_codes), _p(b.Q.c2), _p(b.Q.mean),
+                           _p(b.A), _p(b.B), b.r, ctypes.c_float(b.s), _p(b.y), _p(b.t), _p(b.ws_f),
+                           b.ws_f.numel(), st), "fwd")
+    if ev:
+        q.set_timing_events(ev["bwd"])
+    chk(L.qlora_linear_bwd(_p(b.dY), _p(b.x), _p(b.t), b.M, b.K, b.N, _p(b.Q.codes), _p(b.Q.scale_codes),
+                           _p(b.Q.c2), _p(b.Q.mean), _p(b.A), _p(b.B), b.r, ctypes.c_float(b.s), _p(b.dX),
+                           _p(b.dA), _p(b.dB), _p(b.ws_b), b.ws_b.numel(), st), "bwd")
+    if ev:
+        q.set_timing_events(None)
+
+
+def make_events(n_linears):
+    import torch
+    E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    return [{"q0": E(), "q1": E(), "d1": E(), "fwd": [E() for _ in range(3)], "bwd": [E() for _ in range(6)]}
+            for _ in range(n_linears)]
+
+
+def ours(args, rank, world, dev_index):
+    import torch
+    import bit_nf4_quantized_dq_b200 as q
+
+    dev = torch.device("cuda", dev_index)
+    torch.cuda.set_device(dev)
+    L = q.lib()
+    lins = linears()
+    bufs = [LinearBufs(l, M_TOKENS, R, 3000 + 100 * rank + i, dev) for i, l in enumerate(lins)]
+    wdq = torch.empty(max(l.N * l.K for l in lins), dtype=torch.bfloat16, device=dev)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+
+    def allreduce_grads(b):
+        if dist is not None:
+            dist.all_reduce(b.dA)
+            dist.all_reduce(b.dB)
+
+    stream = torch.cuda.current_stream().cuda_stream
+
+    def step(evs=None):
+        for i, b in enumerate(bufs):
+            run_linear(L, b, wdq, stream, evs[i] if evs else None)
+            allreduce_grads(b)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    q.check_device_error()
+
+    # ------------------------------------------------ device-timed run (inputs resident in HBM)
+    ev_steps = [make_events(len(bufs)) for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(dev_index)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t0.record()
+    for k in range(args.steps):
+        step(ev_steps[k])
+    t1.record()
+    torch.cuda.synchronize()
+    clock_info = clocks.stop()
+    if dist is not None:
+        dist.barrier()
+    q.check_device_error()
+    elapsed_ms = t0.elapsed_time(t1)
+    if dist is not None:
+        tt = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(tt.item())
+    ms_per_step = elapsed_ms / args.steps
+
+    # per-stage totals over the timed steps
+    acc = {k: 0.0 for k in ("quantize", "dequant", "fwd_down", "fwd_fused", "bwd_prep", "bwd_up", "dx_fused",
+                            "dA", "dB")}
+    for evs in ev_steps:
+        for e in evs:
+            acc["quantize"] += e["q0"].elapsed_time(e["q1"])
+            acc["dequant"] += e["q1"].elapsed_time(e["d1"])
+            f, b = e["fwd"], e["bwd"]
+            acc["fwd_down"] += f[0].elapsed_time(f[1])
+            acc["fwd_fused"] += f[1].elapsed_time(f[2])
+            acc["bwd_prep"] += b[0].elapsed_time(b[1])
+            acc["bwd_up"] += b[1].elapsed_time(b[2])
+            acc["dx_fused"] += b[2].elapsed_time(b[3])
+            acc["dA"] += b[3].elapsed_time(b[4])
+            acc["dB"] += b[4].elapsed_time(b[5])
+    K = args.steps
+    weights = sum(l.N * l.K for l in lins)
+    fused_fwd_flops = sum(2 * M_TOKENS * l.N * l.K + 2 * M_TOKENS * l.N * R for l in lins)
+    fused_dx_flops = sum(2 * M_TOKENS * l.N * l.K + 2 * M_TOKENS * l.K * R for l in lins)
+    peaks, peak_src = load_peaks()
+    rows = {
+        "quantize_gbs": weights * CODEC_BYTES_PER_WEIGHT * K / (acc["quantize"] * 1e6),
+        "dequant_gbs": weights * (CODEC_BYTES_PER_WEIGHT) * K / (acc["dequant"] * 1e6),
+        "fwd_fused_tflops": fused_fwd_flops * K / (acc["fwd_fused"] * 1e9),
+        "dx_fused_tflops": fused_dx_flops * K / (acc["dx_fused"] * 1e9),
+        "ms_per_step_by_stage": {k: v / K for k, v in acc.items()},
+    }
+    rows["quantize_frac_hbm"] = rows["quantize_gbs"] / peaks["hbm_gbs"]
+    rows["dequant_frac_hbm"] = rows["dequant_gbs"] / peaks["hbm_gbs"]
+    # dominant kernel: the fused dequant GEMM with the larger total time
+    if acc["fwd_fused"] >= acc["dx_fused"]:
+        dom, dom_flops, dom_ms = "fused forward GEMM (NF4 dequant producer + tcgen05)", fused_fwd_flops, acc["fwd_fused"]
+    else:
+        dom, dom_flops, dom_ms = "fused dX GEMM (NF4 dequant producer + tcgen05)", fused_dx_flops, acc["dx_fused"]
+    launches_per_linear = [b.plan["fwd_launches"] + b.plan["bwd_launches"] + 4 + 1 for b in bufs]
+    achieved = dom_flops / (dom_ms / K) / 1e9
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peaks["bf16_tflops_sustained"],
+                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops_sustained"],
+                "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step)",
+                "traffic": None, "launches_per_step": len(lins), "avg_launch_ms": dom_ms / K / len(lins)}
+
+    # ------------------------------------------------ end to end through host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e = end_to_end(args, bufs, wdq, L, stream, dist, dev)
+
+    flops_all = step_flops() * world
+    value = flops_all / (ms_per_step / 1e3) / 1e12
+    out = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "model": "LLaMA-13B decoder block, 7 linears (random init)",
+                   "tokens_per_gpu": M_TOKENS, "global_batch_tokens": M_TOKENS * world, "r": R, "alpha": ALPHA,
+                   "parallelism": f"dp{world}", "l2": "inputs larger than L2 (weights + activations, about 3 GB)",
+                   "step": "per linear: quantize W, dequant W, fused fwd, bwd (dX, dA, dB)"},
+        "rows": rows, "roofline": roofline, "gpu_launches": sum(launches_per_linear) * K, "clocks": clock_info,
+    }
+    if e2e is not None:
+        out["e2e"] = e2e
+    return out
+
+
+def end_to_end(args, bufs, wdq, L, stream, dist, dev):
+    """Same step through the C ABI with pinned host inputs / outputs copied every step."""
+    import torch
+    host_in, host_out = [], []
+    h2d = d2h = 0
+    for b in bufs:
+        hi = {k: getattr(b, k).to("cpu").pin_memory() for k in ("W", "x", "A", "B", "dY")}
+        ho = {k: torch.empty(getattr(b, k).shape, dtype=getattr(b, k).dtype, pin_memory=True)
+              for k in ("y", "dX", "dA", "dB")}
+        host_in.append(hi)
+        host_out.append(ho)
+        h2d += sum(v.numel() * v.element_size() for v in hi.values())
+        d2h += sum(v.numel() * v.element_size() for v in ho.values())
+
+    def step():
+        for b, hi, ho in zip(bufs, host_in, host_out):
+            for k, v in hi.items():
+                getattr(b, k).copy_(v, non_blocking=True)
+            run_linear(L, b, wdq, stream)
+            if dist is not None:
+                dist.all_reduce(b.dA)
+                dist.all_reduce(b.dB)
+            for k, v in ho.items():
+                v.copy_(getattr(b, k), non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0.record()
+    for _ in range(args.steps):
+        step()
+    t1.record()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1)
+    if dist is not None:
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    world = dist.get_world_size() if dist is not None else 1
+    value = step_flops() * world / (ms / args.steps / 1e3) / 1e12
+    return {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": ms / args.steps}
+
+
+# ------------------------------------------------------------------------------------------
+# the CPU oracle on a bounded sample of the same workload
+# ------------------------------------------------------------------------------------------
+def oracle_sample(codec_weights=1 << 21, tokens=128):
+    """Time the oracle on a sample: the codec (quantize + dequant) on `codec_weights` weights of
+    each linear's weight, and the linear forward + backward of every linear on `tokens` tokens.
+    The per-step time is extrapolated linearly in weights (codec) and in tokens (linear)."""
+    import numpy as np
+    import torch
+    import synth
+    from oracle import linear as olin
+    from oracle import nf4 as onf4
+
+    t_codec = t_lin = 0.0
+    codec_done = 0
+    lin_flops = 0
+    for i, l in enumerate(linears()):
+        W = synth.normal_bf16((l.N, l.K), 0.02, 3000 + i).float().numpy()
+        sub = W.ravel()[:codec_weights]
+        c0 = time.perf_counter()
+        qd = onf4.quantize_nf4_dq(sub)
+        onf4.dequant_nf4_dq(qd["codes"], qd["scale_codes"], qd["c2"], qd["mean"], sub.size)
+        t_codec += time.perf_counter() - c0
+        codec_done += sub.size
+        inp = synth.linear_inputs(tokens, l.N, l.K, R, 3000 + i)
+        f64 = lambda t: t.float().numpy().astype(np.float64)  # noqa: E731
+        x, A, B, dY = (f64(inp[k]) for k in ("x", "A", "B", "dY"))
+        Wd = W.astype(np.float64)          # stands in for W' (same shape; the codec is timed above)
+        c0 = time.perf_counter()
+        olin.qlora_forward(x, Wd, A, B, ALPHA / R)
+        olin.qlora_backward(dY, x, Wd, A, B, ALPHA / R)
+        t_lin += time.perf_counter() - c0
+        lin_flops += linear_flops(tokens, l.N, l.K, R)
+    weights = sum(l.N * l.K for l in linears())
+    est_step_s = t_codec * (weights / codec_done) + t_lin * (step_flops() / lin_flops)
+    cores = len(os.sched_getaffinity(0))
+    return {
+        "value": step_flops() / est_step_s / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+        "sample": (f"codec on the first {codec_weights} weights of each of the 7 weights, fwd+bwd of all 7 "
+                   f"linears on {tokens} of the 8192 tokens (float64 numpy, BLAS threads = {cores}); "
+                   f"step time extrapolated linearly: {est_step_s:.1f} s"),
+        "measured_s": t_codec + t_lin,
+    }
+
+
+def reference(args, rank, world):
+    if rank != 0:
+        return None
+    for _ in range(args.warmup):
+        oracle_sample(codec_weights=1 << 16, tokens=16)
+    vals, runs = [], []
+    for _ in range(args.steps):
+        r = oracle_sample(codec_weights=1 << 19, tokens=64)
+        vals.append(r["value"])
+        runs.append(r)
+    v = statistics.median(vals)
+    last = runs[-1]
+    ms = step_flops() / (v * 1e12) * 1e3
+    return {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "model": "LLaMA-13B decoder block, 7 linears (random init)",
+                   "tokens_per_gpu": M_TOKENS, "r": R, "alpha": ALPHA, "parallelism": "oracle on host cores"},
+        "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": last["cores"], "kind": "oracle",
+                         "sample": last["sample"]},
+        "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end run")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the oracle sample")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        print("note: fewer than 3 warm-up steps", file=sys.stderr)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        out = reference(args, rank, world)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+
+    import torch
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    try:
+        out = ours(args, rank, world, local)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            cb = oracle_sample()
+            out["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

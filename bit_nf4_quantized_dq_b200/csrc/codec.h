@@ -1,0 +1,16 @@
+// Host-side launchers of the NF4 + double-quantization codec kernels.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace qnf4 {
+
+cudaError_t launch_quantize(const uint16_t* W, int64_t numel, uint8_t* codes, uint8_t* scale_codes, float* c2,
+                            float* mean, float* absmax_ws, double* gsum_ws, cudaStream_t st, int sw_encode);
+cudaError_t launch_dequant(const uint8_t* codes, const uint8_t* scale_codes, const float* c2, const float* mean,
+                           int64_t numel, uint16_t* out, cudaStream_t st);
+cudaError_t launch_e4m3_encode(const float* v, int64_t n, uint8_t* out, int sw, cudaStream_t st);
+cudaError_t read_and_clear_error_word(uint32_t* word, cudaStream_t st);
+
+}  // namespace qnf4

@@ -1,0 +1,488 @@
+// tcgen05 GEMM engine with an on-chip NF4 -> bf16 dequant producer.
+//
+// D[rows x cols] (fp32, in TMEM) = sum over K-loop stretches of A[rows x k] * B[cols x k]^T.
+// The 128-row A side is either loaded by TMA or produced on chip from packed NF4 codes (the
+// dequantized 16-bit weights exist only in shared memory, never in HBM); the B side is a
+// K-major bf16 tile loaded by TMA.  One elected thread issues tcgen05.mma (kind::f16,
+// bf16 x bf16 -> fp32) into a TMEM accumulator; four warps read it back for the epilogue.
+//
+// The method's forward and backward ("QLoRA Paper Breakdown: 4-Bit NormalFloat (NF4), Double
+// Quantization, and Paged Optimizers" (fullstackaihub), section 4) map onto this engine as
+//   y^T  = W' x^T + B t^T            (rows = out features, cols = tokens)
+//   dX^T = W'^T dY^T + A^T u^T       (rows = in features,  cols = tokens)
+//   t    = s x A^T,  u = s dY B      (rows = tokens,       cols = rank)
+//   dA^T = x^T u,    dB = dY^T t     (rows = features,     cols = rank, reduced over tokens)
+// with the fp32 intermediates t and u split into bf16 hi + lo parts so that the adapter
+// terms keep close to fp32 accuracy through bf16 tensor-core inputs.
+//
+// Warp roles (192 threads): warp 0 issues TMA loads, warp 1 allocates TMEM and issues MMAs,
+// warps 2-5 run the dequant producer and then the epilogue.
+#pragma once
+
+#include "nf4_device.cuh"
+#include "gemm.h"
+
+namespace qnf4 {
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;
+constexpr int kThreads = 192;
+constexpr int kCodesBytes = 4096;   // packed codes of one 128 x 64 weight tile
+
+template <int BN>
+struct Cfg {
+  static constexpr int kABytes = kBM * kBK * 2;
+  static constexpr int kBBytes = BN * kBK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes + kCodesBytes;
+  static constexpr int kStagesRaw = (220 * 1024 - 2048) / kStageBytes;
+  static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
+  static constexpr int kTmemCols = BN <= 32 ? 32 : BN;
+  static constexpr int kBarrierBytes = 256;
+  static constexpr int kSmemBytes = kStages * kStageBytes + kBarrierBytes + 1024;
+  static_assert(kStages >= 2, "pipeline too shallow");
+  static_assert(kBBytes % 1024 == 0, "B tile must keep 1024-byte alignment");
+};
+
+struct IterPos {
+  int seg;
+  int kb;    // k-block within the stretch
+  bool last; // last k-block of the stretch
+};
+
+// Stretch/k-block of iteration `it` for this CTA: segment 0 restricted to [kb_begin, kb_end),
+// then (split 0 only) every later segment in full.
+__device__ __forceinline__ IterPos iter_pos(const GemmParams& p, int it, int kb_begin, int kb_end, bool first_split) {
+  const int n0 = kb_end - kb_begin;
+  if (it < n0) return IterPos{0, kb_begin + it, kb_begin + it == p.seg[0].kblocks - 1};
+  int rem = it - n0;
+  for (int s = 1; s < p.nseg; ++s) {
+    if (rem < p.seg[s].kblocks) return IterPos{s, rem, rem == p.seg[s].kblocks - 1};
+    rem -= p.seg[s].kblocks;
+  }
+  return IterPos{0, 0, false};
+}
+
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ uint16_t f32_to_bf16_bits(float v) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(v));
+}
+
+// ---------------------------------------------------------------------------------------
+// the dequant producer: one 64-weight unit per thread per k-block
+// ---------------------------------------------------------------------------------------
+// A unit is one (W row n, 64 consecutive W columns) stretch.  It becomes one 128-byte row of
+// the A tile: row t of a K-major tile (forward), or row n_local of MN-major chunk `half`
+// (dX).  16-byte chunk j of the row lands at chunk j ^ (row & 7) (128-byte swizzle).
+struct UnitGeom {
+  int64_t n;      // W row
+  int64_t kcol;   // first W column of the unit
+  uint32_t dst;   // byte offset of the unit's 128-byte row inside the A tile
+  uint32_t swz;   // row & 7
+};
+
+__device__ __forceinline__ UnitGeom unit_geom(int a_src, int t, int row0, int64_t n_base) {
+  UnitGeom u;
+  if (a_src == kANf4K) {
+    u.n = row0 + t;
+    u.kcol = n_base;                 // for the forward, n_base carries the unit's first column
+    u.dst = (uint32_t)t * 128u;
+    u.swz = (uint32_t)t & 7u;
+  } else {
+    const int nl = t >> 1, half = t & 1;
+    u.n = n_base + nl;
+    u.kcol = (int64_t)row0 + 64 * half;
+    u.dst = (uint32_t)half * 8192u + (uint32_t)nl * 128u;
+    u.swz = (uint32_t)nl & 7u;
+  }
+  return u;
+}
+
+__device__ __forceinline__ float unit_scale(const GemmParams& p, int64_t blk, float mean) {
+  const int64_t nb = (p.nw * p.kw + kB1 - 1) / kB1;
+  if (blk < 0 || blk >= nb) return 0.0f;
+  return dq_block_scale(__ldg(p.scale_codes + blk), __ldg(p.c2 + (blk >> 8)), mean);
+}
+
+__device__ __forceinline__ void store_row_chunks(uint8_t* A, const UnitGeom& u, const uint32_t (&words)[8],
+                                                 const Nf4Lut& L0, const Nf4Lut& L1, int split_word,
+                                                 uint32_t valid_words) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    uint32_t o[4];
+    if ((uint32_t)j < valid_words) {
+      nf4_expand8(words[j], j < split_word ? L0 : L1, o);
+    } else {
+      o[0] = o[1] = o[2] = o[3] = 0u;
+    }
+    const uint32_t off = u.dst + (((uint32_t)j ^ u.swz) << 4);
+    *reinterpret_cast<uint4*>(A + off) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_constant__ GemmParams p) {
+  using C = Cfg<BN>;
+  constexpr int S = C::kStages;
+  extern __shared__ uint8_t smem_dyn[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
+  uint64_t* prod = full + S;
+  uint64_t* empty = prod + S;
+  uint64_t* accfull = empty + S;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accfull + 1);
+  volatile uint32_t* abort_word = tmem_slot + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row0 = blockIdx.x * kBM, col0 = blockIdx.y * BN, split = blockIdx.z;
+  const int kb_begin = split * p.kb_per_split;
+  int kb_end = kb_begin + p.kb_per_split;
+  if (kb_end > p.seg[0].kblocks) kb_end = p.seg[0].kblocks;
+  const bool first_split = (split == 0);
+  int n_iters = kb_end - kb_begin;
+  if (first_split)
+    for (int s = 1; s < p.nseg; ++s) n_iters += p.seg[s].kblocks;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&prod[s], 4);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(accfull, 1);
+    *abort_word = 0u;
+    mbar_fence_init();
+  }
+  if (warp == 0 && lane == 0) {
+    for (int m = 0; m < kMaxMaps; ++m) tma_prefetch_desc(&p.maps[m]);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_acc = *tmem_slot;
+
+  auto stage_a = [&](int s) { return smem + s * C::kStageBytes; };
+  auto stage_b = [&](int s) { return smem + s * C::kStageBytes + C::kABytes; };
+  auto stage_c = [&](int s) { return smem + s * C::kStageBytes + C::kABytes + C::kBBytes; };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    int last_issue[8];
+    for (int s = 0; s < 8; ++s) last_issue[s] = -1;
+    bool ok = true;
+    for (int it = 0; it < n_iters && ok; ++it) {
+      const int s = it % S;
+      const uint32_t ph = (uint32_t)(it / S) & 1u;
+      if (!mbar_wait(&empty[s], ph ^ 1u, abort_word, kErrWaitEmpty)) { ok = false; break; }
+      const IterPos ip = iter_pos(p, it, kb_begin, kb_end, first_split);
+      const GemmSeg& sg = p.seg[ip.seg];
+      if (lane == 0) {
+        uint32_t bytes = C::kBBytes;
+        const bool nf4 = (sg.a_src == kANf4K || sg.a_src == kANf4MN);
+        if (nf4 && !p.nf4_generic) bytes += kCodesBytes;
+        if (!nf4) bytes += C::kABytes;
+        mbar_arrive_expect_tx(&full[s], bytes);
+        const int k = sg.a_k0 + ip.kb * kBK;
+        if (sg.a_src == kANf4K) {
+          if (!p.nf4_generic) tma_load_2d(stage_c(s), &p.maps[sg.a_map], k / 2, row0, &full[s]);
+        } else if (sg.a_src == kANf4MN) {
+          if (!p.nf4_generic) tma_load_2d(stage_c(s), &p.maps[sg.a_map], row0 / 2, k, &full[s]);
+        } else if (sg.a_src == kATmaK) {
+          tma_load_2d(stage_a(s), &p.maps[sg.a_map], k, row0, &full[s]);
+        } else {
+          tma_load_2d(stage_a(s), &p.maps[sg.a_map], row0, k, &full[s]);
+          tma_load_2d(stage_a(s) + 8192, &p.maps[sg.a_map], row0 + 64, k, &full[s]);
+        }
+        tma_load_2d(stage_b(s), &p.maps[sg.b_map], sg.b_k0 + ip.kb * kBK, col0, &full[s]);
+        last_issue[s] = it;
+      }
+      __syncwarp();
+    }
+    if (!ok && lane == 0) {
+      // drain copies still in flight before the CTA's shared memory goes away
+      for (int s = 0; s < S; ++s)
+        if (last_issue[s] >= 0) {
+          const uint32_t ph = (uint32_t)(last_issue[s] / S) & 1u;
+          for (int i = 0; i < (1 << 20) && !mbar_try_wait(&full[s], ph); ++i) {}
+        }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    bool ok = true;
+    for (int it = 0; it < n_iters && ok; ++it) {
+      const int s = it % S;
+      const uint32_t ph = (uint32_t)(it / S) & 1u;
+      if (!mbar_wait(&full[s], ph, abort_word, kErrWaitTma)) { ok = false; break; }
+      if (p.has_nf4 && !mbar_wait(&prod[s], ph, abort_word, kErrWaitProducer)) { ok = false; break; }
+      tc_fence_after();
+      const IterPos ip = iter_pos(p, it, kb_begin, kb_end, first_split);
+      const GemmSeg& sg = p.seg[ip.seg];
+      if (lane == 0) {
+        const bool a_mn = (sg.a_src == kANf4MN || sg.a_src == kATmaMN);
+        const uint32_t idesc = umma_idesc_bf16(kBM, BN, a_mn ? 1u : 0u, 0u);
+        const uint32_t a_addr = smem_u32(stage_a(s));
+        const uint32_t b_addr = smem_u32(stage_b(s));
+        const int nk16 = ip.last ? sg.k16_last : 4;
+        for (int k16 = 0; k16 < nk16; ++k16) {
+          const uint64_t ad = a_mn ? umma_sdesc_sw128(a_addr + (uint32_t)k16 * 2048u, 8192u, 1024u)
+                                   : umma_sdesc_sw128(a_addr + (uint32_t)k16 * 32u, 16u, 1024u);
+          const uint64_t bd = umma_sdesc_sw128(b_addr + (uint32_t)k16 * 32u, 16u, 1024u);
+          umma_bf16(tmem_acc, ad, bd, idesc, (it > 0 || k16 > 0) ? 1u : 0u);
+        }
+        umma_commit(&empty[s]);
+      }
+      __syncwarp();
+    }
+    if (lane == 0) umma_commit(accfull);   // also on abort: lets the epilogue wait out in-flight MMAs
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------ dequant producer
+    const int t = threadIdx.x - 64;   // 0..127
+    bool ok = true;
+    if (p.has_nf4) {
+      const float mean = __ldg(p.mean);
+      for (int it = 0; it < n_iters && ok; ++it) {
+        const int s = it % S;
+        const uint32_t ph = (uint32_t)(it / S) & 1u;
+        const IterPos ip = iter_pos(p, it, kb_begin, kb_end, first_split);
+        const GemmSeg& sg = p.seg[ip.seg];
+        const bool nf4 = (sg.a_src == kANf4K || sg.a_src == kANf4MN);
+        UnitGeom u{};
+        Nf4Lut L0, L1;
+        int split_word = 8;
+        uint32_t valid_words = 8;
+        uint32_t words[8];
+        if (nf4) {
+          const int64_t k = (int64_t)sg.a_k0 + (int64_t)ip.kb * kBK;
+          u = unit_geom(sg.a_src, t, row0, k);
+          const bool in_range = (u.n < p.nw) && (u.kcol < p.kw);
+          const int64_t f0 = u.n * p.kw + u.kcol;            // flat index of the unit's first weight
+          const int64_t blk0 = f0 >> 6;
+          float s0 = 0.0f, s1 = 0.0f;
+          if (in_range) {
+            s0 = unit_scale(p, blk0, mean);
+            if (p.nf4_generic) {
+              split_word = (int)((64 - (f0 & 63)) >> 3);     // words before the block boundary
+              if (split_word < 8) s1 = unit_scale(p, blk0 + 1, mean);
+              int64_t vw = (p.kw - u.kcol) >> 3;
+              valid_words = (uint32_t)(vw < 8 ? vw : 8);
+              const uint32_t* src = reinterpret_cast<const uint32_t*>(p.codes + (f0 >> 1));
+#pragma unroll
+              for (int j = 0; j < 8; ++j) words[j] = ((uint32_t)j < valid_words) ? __ldg(src + j) : 0u;
+            }
+          } else {
+            valid_words = 0;
+          }
+          nf4_lut_build(s0, L0);
+          if (split_word < 8) nf4_lut_build(s1, L1);
+          else L1 = L0;
+        }
+        if (!mbar_wait(&full[s], ph, abort_word, kErrWaitTma)) { ok = false; break; }
+        if (nf4) {
+          if (!p.nf4_generic) {
+            const uint4* src = reinterpret_cast<const uint4*>(stage_c(s) + t * 32);
+            const uint4 c0 = src[0], c1 = src[1];
+            words[0] = c0.x; words[1] = c0.y; words[2] = c0.z; words[3] = c0.w;
+            words[4] = c1.x; words[5] = c1.y; words[6] = c1.z; words[7] = c1.w;
+          }
+          store_row_chunks(stage_a(s), u, words, L0, L1, split_word, valid_words);
+          fence_proxy_async_smem();
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&prod[s]);
+      }
+    }
+    // ------------------------------------------------------------------ epilogue
+    if (mbar_wait(accfull, 0u, abort_word, kErrWaitMma)) {
+      tc_fence_after();
+      const int q = warp & 3;
+      const int row = row0 + 32 * q + lane;
+      const bool row_ok = row < p.rows;
+      constexpr int kChunk = BN < 32 ? BN : 32;
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += kChunk) {
+        uint32_t r[32];
+        const uint32_t taddr = tmem_acc + ((uint32_t)(32 * q) << 16) + (uint32_t)c0;
+        if constexpr (kChunk == 32) tmem_ld_32x32b_x32(taddr, r);
+        else tmem_ld_32x32b_x16(taddr, r);
+        tmem_ld_wait();
+        if (!row_ok) continue;
+        if (p.epi == kEpiBf16T) {
+          uint16_t* out = reinterpret_cast<uint16_t*>(p.out);
+#pragma unroll
+          for (int j = 0; j < kChunk; ++j) {
+            const int col = col0 + c0 + j;
+            if (col < p.cols) out[(int64_t)col * p.ld_out + row] = f32_to_bf16_bits(__uint_as_float(r[j]));
+          }
+        } else if (p.epi == kEpiF32T) {
+          float* out = reinterpret_cast<float*>(p.out) + (int64_t)split * p.split_stride;
+#pragma unroll
+          for (int j = 0; j < kChunk; ++j) {
+            const int col = col0 + c0 + j;
+            if (col < p.cols) out[(int64_t)col * p.ld_out + row] = __uint_as_float(r[j]);
+          }
+        } else {
+          float* tout = reinterpret_cast<float*>(p.out);
+#pragma unroll
+          for (int j = 0; j < kChunk; ++j) {
+            const int col = col0 + c0 + j;
+            if (col >= p.cols) continue;
+            const float tv = p.alpha * __uint_as_float(r[j]);
+            const __nv_bfloat16 h = __float2bfloat16_rn(tv);
+            const __nv_bfloat16 l = __float2bfloat16_rn(tv - __bfloat162float(h));
+            if (tout) tout[(int64_t)row * p.ld_out + col] = tv;
+            if (p.hi) p.hi[(int64_t)row * p.ld_hl + col] = __bfloat16_as_ushort(h);
+            if (p.lo) p.lo[(int64_t)row * p.ld_hl + col] = __bfloat16_as_ushort(l);
+            if (p.hiT) p.hiT[(int64_t)col * p.ld_T + row] = __bfloat16_as_ushort(h);
+            if (p.loT) p.loT[(int64_t)col * p.ld_T + row] = __bfloat16_as_ushort(l);
+          }
+        }
+      }
+    }
+    tc_fence_before();
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_acc, C::kTmemCols);
+  }
+}
+
+template <int BN>
+static cudaError_t launch_bn(const GemmParams& p, cudaStream_t st) {
+  using C = Cfg<BN>;
+  static bool configured = false;   // per process; the attribute is per function, not per device
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(qlora_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  dim3 grid((p.rows + kBM - 1) / kBM, (p.cols + BN - 1) / BN, p.splits);
+  qlora_gemm_kernel<BN><<<grid, kThreads, C::kSmemBytes, st>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm(const GemmParams& p, int bn, cudaStream_t st) {
+  switch (bn) {
+    case 16: return launch_bn<16>(p, st);
+    case 32: return launch_bn<32>(p, st);
+    case 64: return launch_bn<64>(p, st);
+    case 128: return launch_bn<128>(p, st);
+    case 256: return launch_bn<256>(p, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// small helpers of the low-rank path
+// ---------------------------------------------------------------------------------------
+// out[c][r] = in[r][c] (bf16), 32x32 tiles through shared memory.
+__global__ void transpose_bf16_kernel(const uint16_t* __restrict__ in, int64_t rows, int64_t cols,
+                                      uint16_t* __restrict__ out, int64_t ld_out) {
+  __shared__ uint16_t tile[32][33];
+  const int64_t r0 = (int64_t)blockIdx.y * 32, c0 = (int64_t)blockIdx.x * 32;
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int64_t r = r0 + i, c = c0 + threadIdx.x;
+    if (r < rows && c < cols) tile[i][threadIdx.x] = in[r * cols + c];
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int64_t c = c0 + i, r = r0 + threadIdx.x;
+    if (r < rows && c < cols) out[c * ld_out + r] = tile[threadIdx.x][i];
+  }
+}
+
+// t [M][r] fp32 -> outT[j][m] = bf16(t), outT[r + j][m] = bf16(t - bf16(t)).
+__global__ void split_hilo_T_kernel(const float* __restrict__ t, int64_t M, int64_t r, uint16_t* __restrict__ outT,
+                                    int64_t ldT) {
+  __shared__ float tile[32][33];
+  const int64_t m0 = (int64_t)blockIdx.y * 32, j0 = (int64_t)blockIdx.x * 32;
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int64_t m = m0 + i, j = j0 + threadIdx.x;
+    tile[i][threadIdx.x] = (m < M && j < r) ? t[m * r + j] : 0.0f;
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int64_t j = j0 + i, m = m0 + threadIdx.x;
+    if (m < M && j < r) {
+      const float v = tile[threadIdx.x][i];
+      const __nv_bfloat16 h = __float2bfloat16_rn(v);
+      outT[j * ldT + m] = __bfloat16_as_ushort(h);
+      outT[(r + j) * ldT + m] = __bfloat16_as_ushort(__float2bfloat16_rn(v - __bfloat162float(h)));
+    }
+  }
+}
+
+// out[c * ld_out + r] = bf16(sum_z ws[z * split_stride + c * ld + r])
+__global__ void reduce_splits_bf16_kernel(const float* __restrict__ ws, int splits, int64_t split_stride,
+                                          int64_t cols, int64_t rows, int64_t ld, uint16_t* __restrict__ out,
+                                          int64_t ld_out) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= cols * rows) return;
+  const int64_t c = i / rows, r = i % rows;
+  float acc = 0.0f;
+  for (int z = 0; z < splits; ++z) acc += ws[(int64_t)z * split_stride + c * ld + r];
+  out[c * ld_out + r] = f32_to_bf16_bits(acc);
+}
+
+// Adapter gradient from hi/lo partials: g[j][i] = sum_z (ws[z][j][i] + ws[z][r + j][i]) for
+// j < r, i < n.  transpose_out = 0 writes out[j * n + i], 1 writes out[i * r + j].
+__global__ void reduce_hilo_kernel(const float* __restrict__ ws, int splits, int64_t split_stride, int64_t r,
+                                   int64_t n, int64_t ld, uint16_t* __restrict__ out, int transpose_out) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= r * n) return;
+  int64_t j, i;
+  if (transpose_out) { i = idx / r; j = idx % r; }
+  else { j = idx / n; i = idx % n; }
+  float acc = 0.0f;
+  for (int z = 0; z < splits; ++z) {
+    const float* w = ws + (int64_t)z * split_stride;
+    acc += w[j * ld + i] + w[(r + j) * ld + i];
+  }
+  out[idx] = f32_to_bf16_bits(acc);
+}
+
+cudaError_t launch_transpose_bf16(const uint16_t* in, int64_t rows, int64_t cols, uint16_t* out, int64_t ld_out,
+                                  cudaStream_t st) {
+  dim3 grid((unsigned)((cols + 31) / 32), (unsigned)((rows + 31) / 32));
+  transpose_bf16_kernel<<<grid, dim3(32, 8), 0, st>>>(in, rows, cols, out, ld_out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_split_hilo_T(const float* t, int64_t M, int64_t r, uint16_t* outT, int64_t ldT, cudaStream_t st) {
+  dim3 grid((unsigned)((r + 31) / 32), (unsigned)((M + 31) / 32));
+  split_hilo_T_kernel<<<grid, dim3(32, 8), 0, st>>>(t, M, r, outT, ldT);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_reduce_splits_bf16(const float* ws, int splits, int64_t split_stride, int64_t cols, int64_t rows,
+                                      int64_t ld, uint16_t* out, int64_t ld_out, cudaStream_t st) {
+  const int64_t n = cols * rows;
+  reduce_splits_bf16_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(ws, splits, split_stride, cols, rows, ld,
+                                                                          out, ld_out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_reduce_hilo(const float* ws, int splits, int64_t split_stride, int64_t r, int64_t n, int64_t ld,
+                               uint16_t* out, int transpose_out, cudaStream_t st) {
+  const int64_t total = r * n;
+  reduce_hilo_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(ws, splits, split_stride, r, n, ld, out,
+                                                                       transpose_out);
+  return cudaGetLastError();
+}
+
+}  // namespace qnf4

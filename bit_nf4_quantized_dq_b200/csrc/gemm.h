@@ -1,0 +1,77 @@
+// Host-side description of one launch of the tcgen05 GEMM engine.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace qnf4 {
+
+// Source of the A operand (the 128-row UMMA "M" side) for one stretch of the K loop.
+enum ASrc : int32_t {
+  kATmaK = 0,    // bf16 tile loaded by TMA, K-major
+  kATmaMN = 1,   // bf16 tile loaded by TMA, MN-major (two 64-wide boxes)
+  kANf4K = 2,    // dequantized on chip from NF4 codes, W rows are the M side (forward)
+  kANf4MN = 3,   // dequantized on chip from NF4 codes, W columns are the M side (dX)
+};
+
+enum Epi : int32_t {
+  kEpiBf16T = 0,    // out_bf16[col * ld + row] = bf16(D[row][col])
+  kEpiF32T = 1,     // ws[split * split_stride + col * ld + row] = D[row][col]
+  kEpiRowHiLo = 2,  // t = alpha * D: t_f32[row][col], hi/lo bf16 [row][col] and [col][row]
+};
+
+struct GemmSeg {
+  int32_t kblocks;    // 64-wide k-blocks in this stretch
+  int32_t k16_last;   // 16-wide MMA steps in its last k-block (1..4)
+  int32_t a_src;      // ASrc
+  int32_t a_map;      // tensor map index for A (codes map for NF4 sources)
+  int32_t b_map;      // tensor map index for B (always K-major bf16)
+  int32_t a_k0;       // first k coordinate of this stretch for A (elements, or W row for kANf4MN)
+  int32_t b_k0;       // first k coordinate of this stretch for B (elements)
+  int32_t pad;
+};
+
+constexpr int kMaxMaps = 5;
+constexpr int kMaxSegs = 3;
+
+struct GemmParams {
+  CUtensorMap maps[kMaxMaps];
+  GemmSeg seg[kMaxSegs];
+  int32_t nseg;
+  int32_t rows, cols;            // valid extent of D: rows on the UMMA M side, cols on the N side
+  int32_t splits, kb_per_split;  // segment 0 is split over blockIdx.z; later segments run in split 0
+  int32_t has_nf4, nf4_generic;  // NF4 producer present; codes fetched without TMA (K % 64 != 0)
+  // NF4 operand: codes / scale codes / group constants / mean of W [nw][kw]
+  const uint8_t* codes;
+  const uint8_t* scale_codes;
+  const float* c2;
+  const float* mean;
+  int64_t nw, kw;
+  // epilogue
+  int32_t epi;
+  float alpha;
+  void* out;
+  int64_t ld_out;
+  int64_t split_stride;
+  uint16_t* hi;   // [rows][cols] bf16, ld = ld_hl
+  uint16_t* lo;
+  uint16_t* hiT;  // [cols][rows] bf16, ld = ld_T
+  uint16_t* loT;
+  int64_t ld_hl, ld_T;
+};
+
+// Launch with tile width bn in {16, 32, 64, 128, 256}; grid = (ceil(rows/128), ceil(cols/bn), splits).
+cudaError_t launch_gemm(const GemmParams& p, int bn, cudaStream_t st);
+
+// Small helpers of the low-rank path.
+cudaError_t launch_transpose_bf16(const uint16_t* in, int64_t rows, int64_t cols, uint16_t* out, int64_t ld_out,
+                                  cudaStream_t st);
+cudaError_t launch_split_hilo_T(const float* t, int64_t M, int64_t r, uint16_t* outT, int64_t ldT,
+                                cudaStream_t st);
+cudaError_t launch_reduce_splits_bf16(const float* ws, int splits, int64_t split_stride, int64_t cols, int64_t rows,
+                                      int64_t ld, uint16_t* out, int64_t ld_out, cudaStream_t st);
+cudaError_t launch_reduce_hilo(const float* ws, int splits, int64_t split_stride, int64_t r, int64_t n, int64_t ld,
+                               uint16_t* out, int transpose_out, cudaStream_t st);
+
+}  // namespace qnf4

@@ -1,0 +1,556 @@
+// The library's single translation unit: the codec and GEMM kernels, and the C ABI
+// (argument checks, workspace layout, TMA tensor maps, kernel sequencing).
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "qlora_nf4.h"
+#include "codec.cuh"
+#include "gemm.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+thread_local void* const* g_events = nullptr;
+thread_local int g_n_events = 0;
+
+void mark(int i, cudaStream_t st) {
+  if (g_events && i < g_n_events && g_events[i]) cudaEventRecord(static_cast<cudaEvent_t>(g_events[i]), st);
+}
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(QNF4_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int check_arch() {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  static int cached_dev = -1, cached_major = 0;
+  if (cached_dev != dev) {
+    int major = 0;
+    e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    cached_dev = dev;
+    cached_major = major;
+  }
+  if (cached_major != 10) return fail(QNF4_ERR_ARCH, "device %d is sm_%d0, this library targets sm_100a", dev,
+                                      cached_major);
+  return QNF4_OK;
+}
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// ------------------------------------------------------------------------ tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D map over a row-major [outer][inner] array with row pitch `row_bytes`.
+int make_map(CUtensorMap* m, const void* base, bool bf16, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+             uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(QNF4_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  if (!aligned(base, 16) || row_bytes % 16 != 0)
+    return fail(QNF4_ERR_UNSUPPORTED, "TMA operand needs a 16-byte aligned base and row pitch (pitch %llu)",
+                (unsigned long long)row_bytes);
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+                   const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   bf16 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(QNF4_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return QNF4_OK;
+}
+
+int bn_for(int64_t cols) {
+  if (cols >= 256) return 256;
+  if (cols > 64) return 128;   // 128 columns: fewer wasted MMA columns than 256
+  if (cols > 32) return 64;
+  if (cols > 16) return 32;
+  return 16;
+}
+
+int kblocks(int64_t k) { return (int)((k + 63) / 64); }
+int k16_last(int64_t k) {
+  const int64_t rem = k - 64 * (int64_t)(kblocks(k) - 1);
+  return (int)((rem + 15) / 16);
+}
+
+constexpr int kSms = 148;
+
+// Split of the K loop over blockIdx.z so that small tile grids still cover the SMs.
+// Every split gets at least one k-block: the count is re-derived from the per-split share.
+int choose_splits(int64_t tiles, int kb) {
+  if (tiles >= kSms) return 1;
+  int64_t s = (kSms + tiles - 1) / tiles;
+  const int64_t cap = kb / 4 > 1 ? kb / 4 : 1;
+  if (s > cap) s = cap;
+  if (s < 1) s = 1;
+  const int64_t per = (kb + s - 1) / s;
+  return (int)((kb + per - 1) / per);
+}
+
+// ------------------------------------------------------------------------ shapes
+struct LinearShape {
+  int64_t M, K, N;
+  int r;
+};
+
+int check_linear_shape(const LinearShape& s) {
+  if (s.M <= 0 || s.K <= 0 || s.N <= 0 || s.r <= 0) return fail(QNF4_ERR_INVALID, "sizes must be positive");
+  if (s.K % 8 || s.N % 8) return fail(QNF4_ERR_UNSUPPORTED, "K and N must be multiples of 8 (K=%lld N=%lld)",
+                                      (long long)s.K, (long long)s.N);
+  if (s.r % 8 || s.r > 256) return fail(QNF4_ERR_UNSUPPORTED, "r must be a multiple of 8 in [8, 256] (r=%d)", s.r);
+  if (s.M >= (1ll << 31) || s.K >= (1ll << 31) || s.N >= (1ll << 31) || s.N * s.K >= (1ll << 40))
+    return fail(QNF4_ERR_INVALID, "sizes too large");
+  return QNF4_OK;
+}
+
+int64_t ld8(int64_t m) { return (m + 7) / 8 * 8; }
+
+// Workspace carving: every region 256-byte aligned.
+struct Carver {
+  char* base;
+  size_t off = 0;
+  template <class T>
+  T* take(size_t count) {
+    off = align_up(off, 256);
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off += count * sizeof(T);
+    return p;
+  }
+};
+
+struct FwdPlan {
+  int bn, splits;
+  int bn_t;
+};
+
+FwdPlan plan_fwd(const LinearShape& s) {
+  FwdPlan p;
+  p.bn = bn_for(s.M);
+  const int64_t tiles = ((s.N + 127) / 128) * ((s.M + p.bn - 1) / p.bn);
+  p.splits = choose_splits(tiles, kblocks(s.K));
+  p.bn_t = bn_for(s.r);
+  return p;
+}
+
+struct BwdPlan {
+  int bn, splits;         // dX
+  int bn_u;               // u = s dY B
+  int bn_g, splits_a, splits_b;   // dA / dB
+};
+
+BwdPlan plan_bwd(const LinearShape& s) {
+  BwdPlan p;
+  p.bn = bn_for(s.M);
+  const int64_t tiles = ((s.K + 127) / 128) * ((s.M + p.bn - 1) / p.bn);
+  p.splits = choose_splits(tiles, kblocks(s.N));
+  p.bn_u = bn_for(s.r);
+  p.bn_g = bn_for(2 * s.r);
+  const int64_t cg = (2 * s.r + p.bn_g - 1) / p.bn_g;
+  p.splits_a = choose_splits(((s.K + 127) / 128) * cg, kblocks(s.M));
+  p.splits_b = choose_splits(((s.N + 127) / 128) * cg, kblocks(s.M));
+  return p;
+}
+
+size_t fwd_carve(Carver& c, const LinearShape& s, const FwdPlan& p, uint16_t** thi, uint16_t** tlo, float** part) {
+  *thi = c.take<uint16_t>((size_t)s.M * s.r);
+  *tlo = c.take<uint16_t>((size_t)s.M * s.r);
+  *part = p.splits > 1 ? c.take<float>((size_t)p.splits * s.M * s.N) : nullptr;
+  return c.off;
+}
+
+struct BwdWs {
+  uint16_t *Bt, *uhi, *ulo, *uT, *tT;
+  float *partX, *partA, *partB;
+};
+
+size_t bwd_carve(Carver& c, const LinearShape& s, const BwdPlan& p, BwdWs* w) {
+  const int64_t ldM = ld8(s.M);
+  w->Bt = c.take<uint16_t>((size_t)s.r * s.N);
+  w->uhi = c.take<uint16_t>((size_t)s.M * s.r);
+  w->ulo = c.take<uint16_t>((size_t)s.M * s.r);
+  w->uT = c.take<uint16_t>((size_t)2 * s.r * ldM);
+  w->tT = c.take<uint16_t>((size_t)2 * s.r * ldM);
+  w->partX = p.splits > 1 ? c.take<float>((size_t)p.splits * s.M * s.K) : nullptr;
+  w->partA = c.take<float>((size_t)p.splits_a * 2 * s.r * s.K);
+  w->partB = c.take<float>((size_t)p.splits_b * 2 * s.r * s.N);
+  return c.off;
+}
+
+int nf4_operand(qnf4::GemmParams& gp, const uint8_t* codes, const uint8_t* scale_codes, const float* c2,
+                const float* mean, int64_t N, int64_t K) {
+  gp.has_nf4 = 1;
+  gp.nf4_generic = (K % 64 != 0) ? 1 : 0;
+  gp.codes = codes;
+  gp.scale_codes = scale_codes;
+  gp.c2 = c2;
+  gp.mean = mean;
+  gp.nw = N;
+  gp.kw = K;
+  return QNF4_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int qnf4_version(void) { return 100; }
+
+int qnf4_set_timing_events(void* const* events, int n) {
+  if (n < 0) return fail(QNF4_ERR_INVALID, "n must be >= 0");
+  g_events = (n > 0) ? events : nullptr;
+  g_n_events = (events && n > 0) ? n : 0;
+  return QNF4_OK;
+}
+
+const char* qnf4_last_error(void) { return g_last_error.c_str(); }
+
+int qnf4_device_error(void* stream, uint32_t* word) {
+  if (!word) return fail(QNF4_ERR_INVALID, "word is NULL");
+  cudaError_t e = qnf4::read_and_clear_error_word(word, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+  if (*word) return fail(QNF4_ERR_DEVICE, "a kernel gave up waiting (flags 0x%x)", *word);
+  return QNF4_OK;
+}
+
+size_t nf4_quantize_workspace_bytes(int64_t numel) {
+  if (numel <= 0) return 0;
+  const int64_t nb = (numel + 63) / 64, ng = (nb + 255) / 256;
+  return align_up((size_t)nb * 4, 256) + (size_t)ng * 8;
+}
+
+int nf4_quantize_dq(const uint16_t* W, int64_t numel, uint8_t* codes, uint8_t* scale_codes, float* c2, float* mean,
+                    void* workspace, size_t workspace_bytes, void* stream) {
+  g_last_error.clear();
+  if (!W || !codes || !scale_codes || !c2 || !mean || !workspace) return fail(QNF4_ERR_INVALID, "NULL pointer");
+  if (numel <= 0) return fail(QNF4_ERR_INVALID, "numel must be positive");
+  if (numel > (1ll << 35)) return fail(QNF4_ERR_UNSUPPORTED, "numel above 2^35");
+  if (!aligned(W, 16) || !aligned(codes, 16) || !aligned(scale_codes, 8) || !aligned(workspace, 256))
+    return fail(QNF4_ERR_UNSUPPORTED, "alignment: W and codes 16 B, scale_codes 8 B, workspace 256 B");
+  if (workspace_bytes < nf4_quantize_workspace_bytes(numel))
+    return fail(QNF4_ERR_WORKSPACE, "workspace needs %zu bytes", nf4_quantize_workspace_bytes(numel));
+  if (int rc = check_arch()) return rc;
+  const int64_t nb = (numel + 63) / 64;
+  float* absmax = static_cast<float*>(workspace);
+  double* gsum = reinterpret_cast<double*>(static_cast<char*>(workspace) + align_up((size_t)nb * 4, 256));
+  cudaError_t e = qnf4::launch_quantize(W, numel, codes, scale_codes, c2, mean, absmax, gsum,
+                                        static_cast<cudaStream_t>(stream), 0);
+  if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
+  return QNF4_OK;
+}
+
+int nf4_dequant(const uint8_t* codes, const uint8_t* scale_codes, const float* c2, const float* mean,
+                int64_t numel, uint16_t* W_out, void* stream) {
+  g_last_error.clear();
+  if (!codes || !scale_codes || !c2 || !mean || !W_out) return fail(QNF4_ERR_INVALID, "NULL pointer");
+  if (numel <= 0) return fail(QNF4_ERR_INVALID, "numel must be positive");
+  if (!aligned(codes, 16) || !aligned(W_out, 16)) return fail(QNF4_ERR_UNSUPPORTED, "codes and W_out need 16 B");
+  if (int rc = check_arch()) return rc;
+  cudaError_t e = qnf4::launch_dequant(codes, scale_codes, c2, mean, numel, W_out, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "dequant launch");
+  return QNF4_OK;
+}
+
+int nf4_e4m3_encode(const float* v, int64_t n, uint8_t* out, int mode, void* stream) {
+  g_last_error.clear();
+  if (!v || !out) return fail(QNF4_ERR_INVALID, "NULL pointer");
+  if (n <= 0) return fail(QNF4_ERR_INVALID, "n must be positive");
+  if (mode != 0 && mode != 1) return fail(QNF4_ERR_INVALID, "mode must be 0 or 1");
+  if (int rc = check_arch()) return rc;
+  cudaError_t e = qnf4::launch_e4m3_encode(v, n, out, mode, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "e4m3 launch");
+  return QNF4_OK;
+}
+
+size_t qlora_linear_fwd_workspace_bytes(int64_t M, int64_t K, int64_t N, int r) {
+  LinearShape s{M, K, N, r};
+  if (M <= 0 || K <= 0 || N <= 0 || r <= 0) return 0;
+  Carver c{nullptr};
+  uint16_t *a, *b;
+  float* p;
+  return fwd_carve(c, s, plan_fwd(s), &a, &b, &p);
+}
+
+int qlora_linear_fwd(const uint16_t* x, int64_t M, int64_t K, int64_t N, const uint8_t* codes,
+                     const uint8_t* scale_codes, const float* c2, const float* mean, const uint16_t* A,
+                     const uint16_t* B, int r, float s, uint16_t* y, float* t_saved, void* workspace,
+                     size_t workspace_bytes, void* stream) {
+  g_last_error.clear();
+  if (!x || !codes || !scale_codes || !c2 || !mean || !A || !B || !y || !t_saved || !workspace)
+    return fail(QNF4_ERR_INVALID, "NULL pointer");
+  LinearShape sh{M, K, N, r};
+  if (int rc = check_linear_shape(sh)) return rc;
+  if (!aligned(x, 16) || !aligned(A, 16) || !aligned(B, 16) || !aligned(y, 16) || !aligned(codes, 16) ||
+      !aligned(t_saved, 16) || !aligned(workspace, 256))
+    return fail(QNF4_ERR_UNSUPPORTED, "alignment: operands 16 B, workspace 256 B");
+  const FwdPlan plan = plan_fwd(sh);
+  Carver c{static_cast<char*>(workspace)};
+  uint16_t *thi, *tlo;
+  float* part;
+  const size_t need = fwd_carve(c, sh, plan, &thi, &tlo, &part);
+  if (workspace_bytes < need) return fail(QNF4_ERR_WORKSPACE, "workspace needs %zu bytes", need);
+  if (int rc = check_arch()) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  mark(0, st);
+
+  // 1) t = s x A^T (fp32 to t_saved), hi / lo bf16 parts to the workspace
+  {
+    qnf4::GemmParams gp;
+    memset(&gp, 0, sizeof(gp));
+    if (int rc = make_map(&gp.maps[0], x, true, K, M, K * 2, 64, 128)) return rc;
+    if (int rc = make_map(&gp.maps[1], A, true, K, r, K * 2, 64, plan.bn_t)) return rc;
+    gp.nseg = 1;
+    gp.seg[0] = qnf4::GemmSeg{kblocks(K), k16_last(K), qnf4::kATmaK, 0, 1, 0, 0, 0};
+    gp.rows = (int32_t)M;
+    gp.cols = r;
+    gp.splits = 1;
+    gp.kb_per_split = kblocks(K);
+    gp.epi = qnf4::kEpiRowHiLo;
+    gp.alpha = s;
+    gp.out = t_saved;
+    gp.ld_out = r;
+    gp.hi = thi;
+    gp.lo = tlo;
+    gp.ld_hl = r;
+    cudaError_t e = qnf4::launch_gemm(gp, plan.bn_t, st);
+    if (e != cudaSuccess) return cuda_fail(e, "down-projection launch");
+  }
+  mark(1, st);
+  // 2) y^T = W' x^T + B t_hi^T + B t_lo^T, W' dequantized on chip
+  {
+    qnf4::GemmParams gp;
+    memset(&gp, 0, sizeof(gp));
+    const bool generic = (K % 64 != 0);
+    if (!generic) {
+      if (int rc = make_map(&gp.maps[0], codes, false, K / 2, N, K / 2, 32, 128)) return rc;
+    }
+    if (int rc = make_map(&gp.maps[1], x, true, K, M, K * 2, 64, plan.bn)) return rc;
+    if (int rc = make_map(&gp.maps[2], B, true, r, N, (uint64_t)r * 2, 64, 128)) return rc;
+    if (int rc = make_map(&gp.maps[3], thi, true, r, M, (uint64_t)r * 2, 64, plan.bn)) return rc;
+    if (int rc = make_map(&gp.maps[4], tlo, true, r, M, (uint64_t)r * 2, 64, plan.bn)) return rc;
+    nf4_operand(gp, codes, scale_codes, c2, mean, N, K);
+    gp.nseg = 3;
+    gp.seg[0] = qnf4::GemmSeg{kblocks(K), k16_last(K), qnf4::kANf4K, 0, 1, 0, 0, 0};
+    gp.seg[1] = qnf4::GemmSeg{kblocks(r), k16_last(r), qnf4::kATmaK, 2, 3, 0, 0, 0};
+    gp.seg[2] = qnf4::GemmSeg{kblocks(r), k16_last(r), qnf4::kATmaK, 2, 4, 0, 0, 0};
+    gp.rows = (int32_t)N;
+    gp.cols = (int32_t)M;
+    gp.splits = plan.splits;
+    gp.kb_per_split = (kblocks(K) + plan.splits - 1) / plan.splits;
+    if (plan.splits > 1) {
+      gp.epi = qnf4::kEpiF32T;
+      gp.out = part;
+      gp.ld_out = N;
+      gp.split_stride = M * N;
+    } else {
+      gp.epi = qnf4::kEpiBf16T;
+      gp.out = y;
+      gp.ld_out = N;
+    }
+    cudaError_t e = qnf4::launch_gemm(gp, plan.bn, st);
+    if (e != cudaSuccess) return cuda_fail(e, "fused forward launch");
+    if (plan.splits > 1) {
+      e = qnf4::launch_reduce_splits_bf16(part, plan.splits, M * N, M, N, N, y, N, st);
+      if (e != cudaSuccess) return cuda_fail(e, "split reduce launch");
+    }
+  }
+  mark(2, st);
+  return QNF4_OK;
+}
+
+int qlora_linear_plan(int64_t M, int64_t K, int64_t N, int r, int* fwd_launches, int* bwd_launches,
+                      int* fwd_splits, int* dx_splits) {
+  g_last_error.clear();
+  LinearShape sh{M, K, N, r};
+  if (int rc = check_linear_shape(sh)) return rc;
+  const FwdPlan f = plan_fwd(sh);
+  const BwdPlan b = plan_bwd(sh);
+  if (fwd_launches) *fwd_launches = 2 + (f.splits > 1 ? 1 : 0);
+  if (bwd_launches) *bwd_launches = 8 + (b.splits > 1 ? 1 : 0);
+  if (fwd_splits) *fwd_splits = f.splits;
+  if (dx_splits) *dx_splits = b.splits;
+  return QNF4_OK;
+}
+
+size_t qlora_linear_bwd_workspace_bytes(int64_t M, int64_t K, int64_t N, int r) {
+  LinearShape s{M, K, N, r};
+  if (M <= 0 || K <= 0 || N <= 0 || r <= 0) return 0;
+  Carver c{nullptr};
+  BwdWs w;
+  return bwd_carve(c, s, plan_bwd(s), &w);
+}
+
+int qlora_linear_bwd(const uint16_t* dY, const uint16_t* x, const float* t_saved, int64_t M, int64_t K, int64_t N,
+                     const uint8_t* codes, const uint8_t* scale_codes, const float* c2, const float* mean,
+                     const uint16_t* A, const uint16_t* B, int r, float s, uint16_t* dX, uint16_t* dA,
+                     uint16_t* dB, void* workspace, size_t workspace_bytes, void* stream) {
+  g_last_error.clear();
+  if (!dY || !x || !t_saved || !codes || !scale_codes || !c2 || !mean || !A || !B || !dA || !dB || !workspace)
+    return fail(QNF4_ERR_INVALID, "NULL pointer");
+  LinearShape sh{M, K, N, r};
+  if (int rc = check_linear_shape(sh)) return rc;
+  if (!aligned(dY, 16) || !aligned(x, 16) || !aligned(A, 16) || !aligned(B, 16) || !aligned(codes, 16) ||
+      !aligned(t_saved, 16) || !aligned(dA, 16) || !aligned(dB, 16) || (dX && !aligned(dX, 16)) ||
+      !aligned(workspace, 256))
+    return fail(QNF4_ERR_UNSUPPORTED, "alignment: operands 16 B, workspace 256 B");
+  const BwdPlan plan = plan_bwd(sh);
+  Carver c{static_cast<char*>(workspace)};
+  BwdWs w;
+  const size_t need = bwd_carve(c, sh, plan, &w);
+  if (workspace_bytes < need) return fail(QNF4_ERR_WORKSPACE, "workspace needs %zu bytes", need);
+  if (int rc = check_arch()) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t ldM = ld8(M);
+  cudaError_t e;
+  mark(0, st);
+
+  // 1) B^T [r][N] and t split into transposed hi / lo rows [2r][M]
+  e = qnf4::launch_transpose_bf16(B, N, r, w.Bt, N, st);
+  if (e != cudaSuccess) return cuda_fail(e, "transpose launch");
+  e = qnf4::launch_split_hilo_T(t_saved, M, r, w.tT, ldM, st);
+  if (e != cudaSuccess) return cuda_fail(e, "split launch");
+  mark(1, st);
+
+  // 2) u = s dY B: hi / lo as [M][r] (dX adapter operand) and as [2r][M] (dA operand)
+  {
+    qnf4::GemmParams gp;
+    memset(&gp, 0, sizeof(gp));
+    if (int rc = make_map(&gp.maps[0], dY, true, N, M, N * 2, 64, 128)) return rc;
+    if (int rc = make_map(&gp.maps[1], w.Bt, true, N, r, N * 2, 64, plan.bn_u)) return rc;
+    gp.nseg = 1;
+    gp.seg[0] = qnf4::GemmSeg{kblocks(N), k16_last(N), qnf4::kATmaK, 0, 1, 0, 0, 0};
+    gp.rows = (int32_t)M;
+    gp.cols = r;
+    gp.splits = 1;
+    gp.kb_per_split = kblocks(N);
+    gp.epi = qnf4::kEpiRowHiLo;
+    gp.alpha = s;
+    gp.out = nullptr;
+    gp.hi = w.uhi;
+    gp.lo = w.ulo;
+    gp.ld_hl = r;
+    gp.hiT = w.uT;
+    gp.loT = w.uT + (size_t)r * ldM;
+    gp.ld_T = ldM;
+    e = qnf4::launch_gemm(gp, plan.bn_u, st);
+    if (e != cudaSuccess) return cuda_fail(e, "up-projection launch");
+  }
+  mark(2, st);
+  // 3) dX^T = W'^T dY^T + A^T u_hi^T + A^T u_lo^T
+  if (dX) {
+    qnf4::GemmParams gp;
+    memset(&gp, 0, sizeof(gp));
+    const bool generic = (K % 64 != 0);
+    if (!generic) {
+      if (int rc = make_map(&gp.maps[0], codes, false, K / 2, N, K / 2, 64, 64)) return rc;
+    }
+    if (int rc = make_map(&gp.maps[1], dY, true, N, M, N * 2, 64, plan.bn)) return rc;
+    if (int rc = make_map(&gp.maps[2], A, true, K, r, K * 2, 64, 64)) return rc;
+    if (int rc = make_map(&gp.maps[3], w.uhi, true, r, M, (uint64_t)r * 2, 64, plan.bn)) return rc;
+    if (int rc = make_map(&gp.maps[4], w.ulo, true, r, M, (uint64_t)r * 2, 64, plan.bn)) return rc;
+    nf4_operand(gp, codes, scale_codes, c2, mean, N, K);
+    gp.nseg = 3;
+    gp.seg[0] = qnf4::GemmSeg{kblocks(N), k16_last(N), qnf4::kANf4MN, 0, 1, 0, 0, 0};
+    gp.seg[1] = qnf4::GemmSeg{kblocks(r), k16_last(r), qnf4::kATmaMN, 2, 3, 0, 0, 0};
+    gp.seg[2] = qnf4::GemmSeg{kblocks(r), k16_last(r), qnf4::kATmaMN, 2, 4, 0, 0, 0};
+    gp.rows = (int32_t)K;
+    gp.cols = (int32_t)M;
+    gp.splits = plan.splits;
+    gp.kb_per_split = (kblocks(N) + plan.splits - 1) / plan.splits;
+    if (plan.splits > 1) {
+      gp.epi = qnf4::kEpiF32T;
+      gp.out = w.partX;
+      gp.ld_out = K;
+      gp.split_stride = M * K;
+    } else {
+      gp.epi = qnf4::kEpiBf16T;
+      gp.out = dX;
+      gp.ld_out = K;
+    }
+    e = qnf4::launch_gemm(gp, plan.bn, st);
+    if (e != cudaSuccess) return cuda_fail(e, "fused dX launch");
+    if (plan.splits > 1) {
+      e = qnf4::launch_reduce_splits_bf16(w.partX, plan.splits, M * K, M, K, K, dX, K, st);
+      if (e != cudaSuccess) return cuda_fail(e, "split reduce launch");
+    }
+  }
+  mark(3, st);
+  // 4) dA^T = x^T [u_hi | u_lo]   (rows K, cols 2r, reduced over M)
+  {
+    qnf4::GemmParams gp;
+    memset(&gp, 0, sizeof(gp));
+    if (int rc = make_map(&gp.maps[0], x, true, K, M, K * 2, 64, 64)) return rc;
+    if (int rc = make_map(&gp.maps[1], w.uT, true, M, 2 * r, ldM * 2, 64, plan.bn_g)) return rc;
+    gp.nseg = 1;
+    gp.seg[0] = qnf4::GemmSeg{kblocks(M), k16_last(M), qnf4::kATmaMN, 0, 1, 0, 0, 0};
+    gp.rows = (int32_t)K;
+    gp.cols = 2 * r;
+    gp.splits = plan.splits_a;
+    gp.kb_per_split = (kblocks(M) + plan.splits_a - 1) / plan.splits_a;
+    gp.epi = qnf4::kEpiF32T;
+    gp.out = w.partA;
+    gp.ld_out = K;
+    gp.split_stride = 2 * r * K;
+    e = qnf4::launch_gemm(gp, plan.bn_g, st);
+    if (e != cudaSuccess) return cuda_fail(e, "dA launch");
+    e = qnf4::launch_reduce_hilo(w.partA, plan.splits_a, 2 * r * K, r, K, K, dA, 0, st);
+    if (e != cudaSuccess) return cuda_fail(e, "dA reduce launch");
+  }
+  mark(4, st);
+  // 5) dB = dY^T [t_hi | t_lo]   (rows N, cols 2r, reduced over M)
+  {
+    qnf4::GemmParams gp;
+    memset(&gp, 0, sizeof(gp));
+    if (int rc = make_map(&gp.maps[0], dY, true, N, M, N * 2, 64, 64)) return rc;
+    if (int rc = make_map(&gp.maps[1], w.tT, true, M, 2 * r, ldM * 2, 64, plan.bn_g)) return rc;
+    gp.nseg = 1;
+    gp.seg[0] = qnf4::GemmSeg{kblocks(M), k16_last(M), qnf4::kATmaMN, 0, 1, 0, 0, 0};
+    gp.rows = (int32_t)N;
+    gp.cols = 2 * r;
+    gp.splits = plan.splits_b;
+    gp.kb_per_split = (kblocks(M) + plan.splits_b - 1) / plan.splits_b;
+    gp.epi = qnf4::kEpiF32T;
+    gp.out = w.partB;
+    gp.ld_out = N;
+    gp.split_stride = 2 * r * N;
+    e = qnf4::launch_gemm(gp, plan.bn_g, st);
+    if (e != cudaSuccess) return cuda_fail(e, "dB launch");
+    e = qnf4::launch_reduce_hilo(w.partB, plan.splits_b, 2 * r * N, r, N, N, dB, 1, st);
+    if (e != cudaSuccess) return cuda_fail(e, "dB reduce launch");
+  }
+  mark(5, st);
+  return QNF4_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,170 @@
+/*
+ * qlora_nf4.h -- C ABI of the NF4 + double-quantization codec and the QLoRA linear layer
+ * for NVIDIA B200 (sm_100a).
+ *
+ * The operations follow the method described in:
+ *   [T] "QLoRA Paper Breakdown: 4-Bit NormalFloat (NF4), Double Quantization, and Paged
+ *       Optimizers" (fullstackaihub teardown): section 2 (code book), section 3 (blockwise
+ *       quantization, double quantization), section 4 (forward pass, dequantization helper,
+ *       backward through the frozen base).
+ *   [E] "QLoRA, explained." (vibeengines): method steps 1-5 and the notation list.
+ *
+ * Conventions for every entry point:
+ *  - Every pointer is a DEVICE pointer owned by the caller, except where stated.  The library
+ *    never allocates device memory and keeps no state between calls other than the device
+ *    error word (see qnf4_device_error).
+ *  - bf16 tensors are passed as uint16_t bit patterns, row-major, densely packed.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every call is
+ *    stream-ordered and asynchronous: it returns after enqueueing its kernels.  Device-side
+ *    faults surface at the caller's next synchronisation.
+ *  - Every call returns an int status (QNF4_OK or a negative QNF4_ERR_*); on error nothing
+ *    has been enqueued unless the status is QNF4_ERR_CUDA (a launch failed part-way), and
+ *    qnf4_last_error() returns a human-readable reason (thread-local).
+ *  - Sizes are int64_t element counts; a size <= 0 is QNF4_ERR_INVALID.
+ *
+ * Stored format of a quantized weight W with numel = N*K elements (row-major [N][K]):
+ *  - blocks are flat runs of 64 consecutive elements of the row-major tensor (a block spans
+ *    two rows when K is not a multiple of 64); nb = ceil(numel/64); the last block is
+ *    zero-padded;
+ *  - codes       : uint8[32*nb], two 4-bit NF4 indices per byte, element 2i in the low
+ *                  nibble of byte i ([T] section 3 level 1, [E] step 2);
+ *  - scale_codes : uint8[nb], the block absmax values centred by the tensor's mean, divided
+ *                  by their group constant, as E4M3 8-bit floats ([T] section 3 level 2);
+ *  - c2          : float[ceil(nb/256)], one fp32 constant per group of 256 scale codes;
+ *  - mean        : float[1], the fp32 mean of all block absmax values.
+ * Storage: 4 + 8/64 + 32/(64*256) = 4.126953125 bits per weight, plus 32 bits for the mean.
+ */
+#ifndef QLORA_NF4_H
+#define QLORA_NF4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define QNF4_OK 0
+#define QNF4_ERR_INVALID (-1)     /* null pointer, size <= 0, size overflow */
+#define QNF4_ERR_UNSUPPORTED (-2) /* unsupported shape or alignment (see each call) */
+#define QNF4_ERR_ARCH (-3)        /* current device is not sm_100 */
+#define QNF4_ERR_CUDA (-4)        /* a CUDA call or launch failed; see qnf4_last_error() */
+#define QNF4_ERR_DEVICE (-5)      /* a kernel's bounded wait ran out (device error word set) */
+#define QNF4_ERR_WORKSPACE (-6)   /* workspace too small */
+
+/* Library version (major*10000 + minor*100 + patch). */
+int qnf4_version(void);
+
+/* Reason for the last non-OK status returned on this host thread ("" if none).  The
+ * string is owned by the library and valid until the next call on this thread. */
+const char* qnf4_last_error(void);
+
+/* Synchronises `stream`, then reads and clears the device error word of the current device.
+ * *word receives the bit flags (0 = no kernel gave up waiting).  Returns QNF4_ERR_DEVICE if
+ * the word was non-zero, QNF4_ERR_CUDA if the synchronisation failed.  `word` is a HOST
+ * pointer. */
+int qnf4_device_error(void* stream, uint32_t* word);
+
+/* ---------------------------------------------------------------------------------------
+ * NF4 blockwise quantization with double quantization.
+ * [T] section 3 (both levels), [E] steps 2-3.
+ *
+ *   W           : bf16[numel], read only.
+ *   codes       : uint8[32*nb], written.     16-byte aligned.
+ *   scale_codes : uint8[nb], written.        8-byte aligned.
+ *   c2          : float[ceil(nb/256)], written.
+ *   mean        : float[1], written.
+ *   workspace   : device scratch of at least nf4_quantize_workspace_bytes(numel) bytes,
+ *                 256-byte aligned; its contents are undefined afterwards.
+ * W must be 16-byte aligned.  numel <= 2^35.  Weights must be finite.  Bit-exact with the
+ * method's definition: absmax per block, n = fp32(w / absmax) (correctly rounded), the
+ * nearest code-book level (ties to the lower level; an all-zero block codes to level 7),
+ * mean = fp32(float64 pairwise sum / nb), d = fp32(absmax - mean), c2 = max |d| per group,
+ * scale code = E4M3 round-to-nearest-even of fp32(d / c2) (c2 == 0 gives code 0).
+ * ------------------------------------------------------------------------------------- */
+size_t nf4_quantize_workspace_bytes(int64_t numel);
+int nf4_quantize_dq(const uint16_t* W, int64_t numel, uint8_t* codes, uint8_t* scale_codes, float* c2,
+                    float* mean, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * NF4 + DQ -> bf16 dequantization (the standalone HBM stream).
+ * [T] section 4, dequantization helper; [E] step 4.
+ *
+ *   W_out[e] = bf16_rn( fp32_rn( level[code_e] * s_b ) ),  s_b = fmaf(e4m3(scale_code_b), c2_g, mean)
+ * codes must be 16-byte aligned and W_out 16-byte aligned.  Inputs are read only.
+ * ------------------------------------------------------------------------------------- */
+int nf4_dequant(const uint8_t* codes, const uint8_t* scale_codes, const float* c2, const float* mean,
+                int64_t numel, uint16_t* W_out, void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * QLoRA linear layer, forward.  [T] section 4 (forward pass), [E] steps 4-5.
+ *
+ *   y = x W'^T + s (x A^T) B^T,   W' = dequant(codes, scale_codes, c2, mean)  ([N][K])
+ *
+ *   x       : bf16[M][K]          A : bf16[r][K]          B : bf16[N][r]
+ *   y       : bf16[M][N], written
+ *   t_saved : float[M][r], written: t = s x A^T (fp32), kept by the caller for the backward
+ * W' is produced tile by tile in shared memory from the codes and is never written to HBM.
+ * Requirements: K % 8 == 0, N % 8 == 0, r % 8 == 0, 8 <= r <= 256, bf16 and code pointers
+ * 16-byte aligned.  Accuracy: fp32 accumulation of exact bf16 products; the adapter term uses
+ * t split into bf16 hi + lo parts.  Workspace: qlora_linear_fwd_workspace_bytes(M, K, N, r)
+ * bytes, 256-byte aligned.
+ * ------------------------------------------------------------------------------------- */
+size_t qlora_linear_fwd_workspace_bytes(int64_t M, int64_t K, int64_t N, int r);
+int qlora_linear_fwd(const uint16_t* x, int64_t M, int64_t K, int64_t N, const uint8_t* codes,
+                     const uint8_t* scale_codes, const float* c2, const float* mean, const uint16_t* A,
+                     const uint16_t* B, int r, float s, uint16_t* y, float* t_saved, void* workspace,
+                     size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * QLoRA linear layer, backward.  [T] section 4 (gradients reach the input through the
+ * dequantized frozen base; no gradient of W is formed), [E] step 5 (only the adapters train).
+ *
+ *   u  = s dY B              (fp32, split into bf16 hi + lo)
+ *   dX = dY W' + u A         (W' produced on chip from the codes, transposed operand)
+ *   dA = u^T x               (reduction over the M tokens)
+ *   dB = dY^T t_saved        (t_saved from qlora_linear_fwd on the same x, A and s)
+ *
+ *   dY : bf16[M][N]   x : bf16[M][K]   t_saved : float[M][r]
+ *   dX : bf16[M][K], written (may be NULL to skip)   dA : bf16[r][K]   dB : bf16[N][r]
+ * Same shape / alignment requirements as the forward.  Workspace:
+ * qlora_linear_bwd_workspace_bytes(M, K, N, r) bytes, 256-byte aligned.
+ * ------------------------------------------------------------------------------------- */
+size_t qlora_linear_bwd_workspace_bytes(int64_t M, int64_t K, int64_t N, int r);
+int qlora_linear_bwd(const uint16_t* dY, const uint16_t* x, const float* t_saved, int64_t M, int64_t K, int64_t N,
+                     const uint8_t* codes, const uint8_t* scale_codes, const float* c2, const float* mean,
+                     const uint16_t* A, const uint16_t* B, int r, float s, uint16_t* dX, uint16_t* dA,
+                     uint16_t* dB, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * Launch plan of one forward / backward call of this shape (host-only, no device work):
+ * the number of kernels each call enqueues, and the split factor of the K loop of the
+ * fused dequant GEMMs (1 = no split).  Output pointers are HOST pointers and may be NULL.
+ * ------------------------------------------------------------------------------------- */
+int qlora_linear_plan(int64_t M, int64_t K, int64_t N, int r, int* fwd_launches, int* bwd_launches,
+                      int* fwd_splits, int* dx_splits);
+
+/* ---------------------------------------------------------------------------------------
+ * Optional stage timing (a profiling aid, no counterpart in the method).  When `events`
+ * is non-NULL, later calls made from this host thread record the caller's cudaEvent_t
+ * handles on their stream at stage boundaries (events[i] for i < n only):
+ *   qlora_linear_fwd: [0] start, [1] after the down-projection t = s x A^T, [2] end (after
+ *                     the fused dequant GEMM and its split reduction, if any);
+ *   qlora_linear_bwd: [0] start, [1] after the B transpose and t split, [2] after
+ *                     u = s dY B, [3] after the fused dX GEMM, [4] after dA, [5] end (dB).
+ * The handles stay owned by the caller; pass NULL (or n = 0) to stop recording.
+ * ------------------------------------------------------------------------------------- */
+int qnf4_set_timing_events(void* const* events, int n);
+
+/* ---------------------------------------------------------------------------------------
+ * E4M3 encoding of an fp32 array, as used for the scale codes (round to nearest even,
+ * saturating at 448, sign kept).  mode 0 = hardware conversion (the one nf4_quantize_dq
+ * uses), mode 1 = the library's software encoder.  A utility for checking the format.
+ * ------------------------------------------------------------------------------------- */
+int nf4_e4m3_encode(const float* v, int64_t n, uint8_t* out, int mode, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLORA_NF4_H */

@@ -56,6 +56,15 @@ def qlora_backward(dY, x, w_deq, A, B, s: float) -> dict:
     return {"dX": dX, "dA": dA, "dB": dB, "u": u}
 
 
+def adapter_grads(dY, x, A, B, s: float) -> dict:
+    """dA and dB alone (same definitions as ``qlora_backward``), for shapes where the full
+    dX product is too slow on the host; also returns t = s x A^T."""
+    dY = _f64(dY); x = _f64(x); A = _f64(A); B = _f64(B)
+    s = float(s)
+    xa = x @ A.T
+    return {"dA": (s * (dY @ B)).T @ x, "dB": s * (dY.T @ xa), "t": s * xa}
+
+
 def forward_rows(x, w_deq, A, B, s: float, rows) -> np.ndarray:
     """Rows ``rows`` of y only (for sampled checks at sizes where the full product is slow)."""
     rows = np.asarray(rows)

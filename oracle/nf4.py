@@ -235,6 +235,51 @@ def _fmaf(a: np.ndarray, b: np.ndarray, c: np.ndarray) -> np.ndarray:
 # quantize: steps 2 and 3 of the method
 # ----------------------------------------------------------------------------------------
 
+def block_absmax(w) -> np.ndarray:
+    """Step 1-2 of ``quantize_nf4_dq``: absmax of each flat block of 64 (zero-padded tail)."""
+    w = np.asarray(w, dtype=np.float32).ravel()
+    nb = -(-w.size // B1)
+    wp = np.zeros(nb * B1, dtype=np.float32)
+    wp[:w.size] = w
+    return np.max(np.abs(wp.reshape(nb, B1)), axis=1).astype(np.float32)
+
+
+def level1_codes(w) -> tuple:
+    """Steps 1-4 of ``quantize_nf4_dq``: per-block absmax and the packed NF4 codes."""
+    w = np.asarray(w, dtype=np.float32).ravel()
+    nb = -(-w.size // B1)
+    wp = np.zeros(nb * B1, dtype=np.float32)
+    wp[:w.size] = w
+    blocks = wp.reshape(nb, B1)
+    absmax = np.max(np.abs(blocks), axis=1).astype(np.float32)
+    safe = np.where(absmax > 0, absmax, np.float32(1)).astype(np.float64)
+    n = (blocks.astype(np.float64) / safe[:, None]).astype(np.float32)
+    codes = nearest_level(n).reshape(nb, B1)
+    codes[absmax == 0, :] = 7
+    flat_codes = codes.ravel()
+    packed = (flat_codes[0::2] | (flat_codes[1::2] << 4)).astype(np.uint8)
+    return absmax, packed
+
+
+def double_quantize(absmax) -> dict:
+    """Step 5 of ``quantize_nf4_dq``: mean, group constants c2 and E4M3 scale codes."""
+    absmax = np.asarray(absmax, dtype=np.float32)
+    nb = absmax.size
+    mean = np.float32(np.float64(tree_sum_f64(absmax)) / np.float64(nb))
+    d = (absmax.astype(np.float64) - np.float64(mean)).astype(np.float32)
+    ng = -(-nb // B2)
+    c2 = np.zeros(ng, dtype=np.float32)
+    scale_codes = np.zeros(nb, dtype=np.uint8)
+    for g in range(ng):
+        dg = d[g * B2:(g + 1) * B2]
+        m = np.float32(np.max(np.abs(dg)))
+        c2[g] = m
+        if m > 0:
+            v = (dg.astype(np.float64) / np.float64(m)).astype(np.float32)
+            scale_codes[g * B2:(g + 1) * B2] = e4m3_encode_rn(v)
+    return {"scale_codes": scale_codes, "c2": c2, "mean": np.float32(mean)}
+
+
 def quantize_nf4_dq(w) -> dict:
     """Quantize a weight tensor (given as bf16-exact values) to NF4 codes plus DQ scales.
 
@@ -259,36 +304,12 @@ def quantize_nf4_dq(w) -> dict:
     intermediate ``absmax`` (float32, nb) for inspection.
     """
     w = np.asarray(w, dtype=np.float32).ravel()
-    numel = w.size
-    if numel == 0:
+    if w.size == 0:
         raise ValueError("empty tensor")
-    nb = -(-numel // B1)
-    wp = np.zeros(nb * B1, dtype=np.float32)
-    wp[:numel] = w
-    blocks = wp.reshape(nb, B1)
-
-    absmax = np.max(np.abs(blocks), axis=1).astype(np.float32)
-    safe = np.where(absmax > 0, absmax, np.float32(1)).astype(np.float64)
-    n = (blocks.astype(np.float64) / safe[:, None]).astype(np.float32)
-    codes = nearest_level(n).reshape(nb, B1)
-    codes[absmax == 0, :] = 7
-    flat_codes = codes.ravel()
-    packed = (flat_codes[0::2] | (flat_codes[1::2] << 4)).astype(np.uint8)
-
-    mean = np.float32(np.float64(tree_sum_f64(absmax)) / np.float64(nb))
-    d = (absmax.astype(np.float64) - np.float64(mean)).astype(np.float32)
-    ng = -(-nb // B2)
-    c2 = np.zeros(ng, dtype=np.float32)
-    scale_codes = np.zeros(nb, dtype=np.uint8)
-    for g in range(ng):
-        dg = d[g * B2:(g + 1) * B2]
-        m = np.float32(np.max(np.abs(dg)))
-        c2[g] = m
-        if m > 0:
-            v = (dg.astype(np.float64) / np.float64(m)).astype(np.float32)
-            scale_codes[g * B2:(g + 1) * B2] = e4m3_encode_rn(v)
-    return {"codes": packed, "scale_codes": scale_codes, "c2": c2,
-            "mean": np.float32(mean), "absmax": absmax, "numel": numel}
+    absmax, packed = level1_codes(w)
+    dq = double_quantize(absmax)
+    return {"codes": packed, "scale_codes": dq["scale_codes"], "c2": dq["c2"],
+            "mean": dq["mean"], "absmax": absmax, "numel": w.size}
 
 
 def unpack_codes(packed: np.ndarray, numel: int) -> np.ndarray:

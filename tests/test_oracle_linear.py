@@ -74,5 +74,13 @@ def test_sampled_rows_match_full():
     assert np.allclose(linear.dx_rows(dY, W, A, B, 0.3, rows), g["dX"][rows], atol=1e-13)
 
 
+def test_adapter_grads_match_full_backward():
+    x, W, A, B, dY = _tiny(5, M=8, N=6, K=7, r=3)
+    g = linear.qlora_backward(dY, x, W, A, B, 0.4)
+    a = linear.adapter_grads(dY, x, A, B, 0.4)
+    assert np.allclose(a["dA"], g["dA"], atol=1e-13) and np.allclose(a["dB"], g["dB"], atol=1e-13)
+    assert np.allclose(a["t"], linear.qlora_forward(x, W, A, B, 0.4)["t"], atol=1e-13)
+
+
 def test_flop_count():
     assert linear.linear_flops(2, 3, 5, 7) == 4 * 2 * 3 * 5 + 6 * 2 * 5 * 7 + 6 * 2 * 3 * 7
