@@ -197,8 +197,15 @@ def run_linear(L, b: LinearBufs, wdq, stream, ev=None):
 
 
 def make_events(n_linears):
+    """Timing events of one step.  torch only reports elapsed time between events it has
+    recorded itself, so every event is recorded once here (outside any timed region); the
+    library's stage marks then re-record the same handles at the stage boundaries."""
     import torch
-    E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+
+    def E():
+        e = torch.cuda.Event(enable_timing=True)
+        e.record()
+        return e
     return [{"q0": E(), "q1": E(), "d1": E(), "fwd": [E() for _ in range(3)], "bwd": [E() for _ in range(6)]}
             for _ in range(n_linears)]
 
@@ -216,11 +223,11 @@ def ours(args, rank, world, dev_index):
     dist = None
     if world > 1:
         import torch.distributed as dist
+    from bit_nf4_quantized_dq_b200.dp import allreduce_adapter_grads
 
     def allreduce_grads(b):
         if dist is not None:
-            dist.all_reduce(b.dA)
-            dist.all_reduce(b.dB)
+            allreduce_adapter_grads([b.dA, b.dB])
 
     stream = torch.cuda.current_stream().cuda_stream
 
@@ -324,6 +331,7 @@ def ours(args, rank, world, dev_index):
 def end_to_end(args, bufs, wdq, L, stream, dist, dev):
     """Same step through the C ABI with pinned host inputs / outputs copied every step."""
     import torch
+    from bit_nf4_quantized_dq_b200.dp import allreduce_adapter_grads
     host_in, host_out = [], []
     h2d = d2h = 0
     for b in bufs:
@@ -341,8 +349,7 @@ def end_to_end(args, bufs, wdq, L, stream, dist, dev):
                 getattr(b, k).copy_(v, non_blocking=True)
             run_linear(L, b, wdq, stream)
             if dist is not None:
-                dist.all_reduce(b.dA)
-                dist.all_reduce(b.dB)
+                allreduce_adapter_grads([b.dA, b.dB])
             for k, v in ho.items():
                 v.copy_(getattr(b, k), non_blocking=True)
 
@@ -438,6 +445,61 @@ def reference(args, rank, world):
     }
 
 
+CASES = ("fwd", "bwd", "quantize", "dequant")
+
+
+def single_case(args):
+    """One linear of the block (`--linear`, default q: 5120x5120) at 8192 tokens; runs only the
+    calls of `--case` (after one quantize), `--warmup` + `--steps` times.  Small enough (about
+    0.2-0.6 GB on the device, more than L2) for profiler captures of one kernel family."""
+    import ctypes
+    import torch
+    import bit_nf4_quantized_dq_b200 as q
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    L = q.lib()
+    lin = {l.name: l for l in linears()}[args.linear]
+    b = LinearBufs(lin, M_TOKENS, R, 3000, dev)
+    wdq = torch.empty(lin.N * lin.K, dtype=torch.bfloat16, device=dev)
+    st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    numel = lin.N * lin.K
+
+    def quantize():
+        assert L.nf4_quantize_dq(_p(b.W), numel, _p(b.Q.codes), _p(b.Q.scale_codes), _p(b.Q.c2), _p(b.Q.mean),
+                                 _p(b.ws_q), b.ws_q.numel(), st) == 0
+
+    def fwd():
+        assert L.qlora_linear_fwd(_p(b.x), b.M, b.K, b.N, _p(b.Q.codes), _p(b.Q.scale_codes), _p(b.Q.c2),
+                                  _p(b.Q.mean), _p(b.A), _p(b.B), b.r, ctypes.c_float(b.s), _p(b.y), _p(b.t),
+                                  _p(b.ws_f), b.ws_f.numel(), st) == 0
+
+    def bwd():
+        assert L.qlora_linear_bwd(_p(b.dY), _p(b.x), _p(b.t), b.M, b.K, b.N, _p(b.Q.codes), _p(b.Q.scale_codes),
+                                  _p(b.Q.c2), _p(b.Q.mean), _p(b.A), _p(b.B), b.r, ctypes.c_float(b.s), _p(b.dX),
+                                  _p(b.dA), _p(b.dB), _p(b.ws_b), b.ws_b.numel(), st) == 0
+
+    def dequant():
+        assert L.nf4_dequant(_p(b.Q.codes), _p(b.Q.scale_codes), _p(b.Q.c2), _p(b.Q.mean), numel, _p(wdq), st) == 0
+
+    quantize()
+    if args.case == "bwd":
+        fwd()
+    fn = {"fwd": fwd, "bwd": bwd, "quantize": quantize, "dequant": dequant}[args.case]
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(args.steps):
+        fn()
+    t1.record()
+    torch.cuda.synchronize()
+    q.check_device_error()
+    ms = t0.elapsed_time(t1) / args.steps
+    print(json.dumps({"case": args.case, "linear": args.linear, "tokens": M_TOKENS, "ms_per_call": ms}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -446,7 +508,13 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end run")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the oracle sample")
+    ap.add_argument("--case", choices=CASES, default=None,
+                    help="run one call family on one linear only (profiling aid; prints its own line)")
+    ap.add_argument("--linear", default="q", help="linear of the block used by --case")
     args = ap.parse_args()
+    if args.case:
+        single_case(args)
+        return
     if args.warmup < 3 and args.impl == "ours":
         print("note: fewer than 3 warm-up steps", file=sys.stderr)
 

@@ -333,21 +333,6 @@ __global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_co
             const int col = col0 + c0 + j;
             if (col < p.cols) out[(int64_t)col * p.ld_out + row] = __uint_as_float(r[j]);
           }
-        } else {
-          float* tout = reinterpret_cast<float*>(p.out);
-#pragma unroll
-          for (int j = 0; j < kChunk; ++j) {
-            const int col = col0 + c0 + j;
-            if (col >= p.cols) continue;
-            const float tv = p.alpha * __uint_as_float(r[j]);
-            const __nv_bfloat16 h = __float2bfloat16_rn(tv);
-            const __nv_bfloat16 l = __float2bfloat16_rn(tv - __bfloat162float(h));
-            if (tout) tout[(int64_t)row * p.ld_out + col] = tv;
-            if (p.hi) p.hi[(int64_t)row * p.ld_hl + col] = __bfloat16_as_ushort(h);
-            if (p.lo) p.lo[(int64_t)row * p.ld_hl + col] = __bfloat16_as_ushort(l);
-            if (p.hiT) p.hiT[(int64_t)col * p.ld_T + row] = __bfloat16_as_ushort(h);
-            if (p.loT) p.loT[(int64_t)col * p.ld_T + row] = __bfloat16_as_ushort(l);
-          }
         }
       }
     }
@@ -406,26 +391,6 @@ __global__ void transpose_bf16_kernel(const uint16_t* __restrict__ in, int64_t r
   }
 }
 
-// t [M][r] fp32 -> outT[j][m] = bf16(t), outT[r + j][m] = bf16(t - bf16(t)).
-__global__ void split_hilo_T_kernel(const float* __restrict__ t, int64_t M, int64_t r, uint16_t* __restrict__ outT,
-                                    int64_t ldT) {
-  __shared__ float tile[32][33];
-  const int64_t m0 = (int64_t)blockIdx.y * 32, j0 = (int64_t)blockIdx.x * 32;
-  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
-    const int64_t m = m0 + i, j = j0 + threadIdx.x;
-    tile[i][threadIdx.x] = (m < M && j < r) ? t[m * r + j] : 0.0f;
-  }
-  __syncthreads();
-  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
-    const int64_t j = j0 + i, m = m0 + threadIdx.x;
-    if (m < M && j < r) {
-      const float v = tile[threadIdx.x][i];
-      const __nv_bfloat16 h = __float2bfloat16_rn(v);
-      outT[j * ldT + m] = __bfloat16_as_ushort(h);
-      outT[(r + j) * ldT + m] = __bfloat16_as_ushort(__float2bfloat16_rn(v - __bfloat162float(h)));
-    }
-  }
-}
 
 // out[c * ld_out + r] = bf16(sum_z ws[z * split_stride + c * ld + r])
 __global__ void reduce_splits_bf16_kernel(const float* __restrict__ ws, int splits, int64_t split_stride,
@@ -439,22 +404,6 @@ __global__ void reduce_splits_bf16_kernel(const float* __restrict__ ws, int spli
   out[c * ld_out + r] = f32_to_bf16_bits(acc);
 }
 
-// Adapter gradient from hi/lo partials: g[j][i] = sum_z (ws[z][j][i] + ws[z][r + j][i]) for
-// j < r, i < n.  transpose_out = 0 writes out[j * n + i], 1 writes out[i * r + j].
-__global__ void reduce_hilo_kernel(const float* __restrict__ ws, int splits, int64_t split_stride, int64_t r,
-                                   int64_t n, int64_t ld, uint16_t* __restrict__ out, int transpose_out) {
-  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= r * n) return;
-  int64_t j, i;
-  if (transpose_out) { i = idx / r; j = idx % r; }
-  else { j = idx / n; i = idx % n; }
-  float acc = 0.0f;
-  for (int z = 0; z < splits; ++z) {
-    const float* w = ws + (int64_t)z * split_stride;
-    acc += w[j * ld + i] + w[(r + j) * ld + i];
-  }
-  out[idx] = f32_to_bf16_bits(acc);
-}
 
 cudaError_t launch_transpose_bf16(const uint16_t* in, int64_t rows, int64_t cols, uint16_t* out, int64_t ld_out,
                                   cudaStream_t st) {
@@ -463,11 +412,6 @@ cudaError_t launch_transpose_bf16(const uint16_t* in, int64_t rows, int64_t cols
   return cudaGetLastError();
 }
 
-cudaError_t launch_split_hilo_T(const float* t, int64_t M, int64_t r, uint16_t* outT, int64_t ldT, cudaStream_t st) {
-  dim3 grid((unsigned)((r + 31) / 32), (unsigned)((M + 31) / 32));
-  split_hilo_T_kernel<<<grid, dim3(32, 8), 0, st>>>(t, M, r, outT, ldT);
-  return cudaGetLastError();
-}
 
 cudaError_t launch_reduce_splits_bf16(const float* ws, int splits, int64_t split_stride, int64_t cols, int64_t rows,
                                       int64_t ld, uint16_t* out, int64_t ld_out, cudaStream_t st) {
@@ -477,12 +421,5 @@ cudaError_t launch_reduce_splits_bf16(const float* ws, int splits, int64_t split
   return cudaGetLastError();
 }
 
-cudaError_t launch_reduce_hilo(const float* ws, int splits, int64_t split_stride, int64_t r, int64_t n, int64_t ld,
-                               uint16_t* out, int transpose_out, cudaStream_t st) {
-  const int64_t total = r * n;
-  reduce_hilo_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(ws, splits, split_stride, r, n, ld, out,
-                                                                       transpose_out);
-  return cudaGetLastError();
-}
 
 }  // namespace qnf4

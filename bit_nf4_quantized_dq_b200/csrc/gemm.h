@@ -18,7 +18,6 @@ enum ASrc : int32_t {
 enum Epi : int32_t {
   kEpiBf16T = 0,    // out_bf16[col * ld + row] = bf16(D[row][col])
   kEpiF32T = 1,     // ws[split * split_stride + col * ld + row] = D[row][col]
-  kEpiRowHiLo = 2,  // t = alpha * D: t_f32[row][col], hi/lo bf16 [row][col] and [col][row]
 };
 
 struct GemmSeg {
@@ -54,11 +53,6 @@ struct GemmParams {
   void* out;
   int64_t ld_out;
   int64_t split_stride;
-  uint16_t* hi;   // [rows][cols] bf16, ld = ld_hl
-  uint16_t* lo;
-  uint16_t* hiT;  // [cols][rows] bf16, ld = ld_T
-  uint16_t* loT;
-  int64_t ld_hl, ld_T;
 };
 
 // Launch with tile width bn in {16, 32, 64, 128, 256}; grid = (ceil(rows/128), ceil(cols/bn), splits).
@@ -67,11 +61,7 @@ cudaError_t launch_gemm(const GemmParams& p, int bn, cudaStream_t st);
 // Small helpers of the low-rank path.
 cudaError_t launch_transpose_bf16(const uint16_t* in, int64_t rows, int64_t cols, uint16_t* out, int64_t ld_out,
                                   cudaStream_t st);
-cudaError_t launch_split_hilo_T(const float* t, int64_t M, int64_t r, uint16_t* outT, int64_t ldT,
-                                cudaStream_t st);
 cudaError_t launch_reduce_splits_bf16(const float* ws, int splits, int64_t split_stride, int64_t cols, int64_t rows,
                                       int64_t ld, uint16_t* out, int64_t ld_out, cudaStream_t st);
-cudaError_t launch_reduce_hilo(const float* ws, int splits, int64_t split_stride, int64_t r, int64_t n, int64_t ld,
-                               uint16_t* out, int transpose_out, cudaStream_t st);
 
 }  // namespace qnf4

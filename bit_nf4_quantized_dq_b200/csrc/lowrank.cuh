@@ -1,0 +1,353 @@
+// Low-rank products of the QLoRA linear with float64-accurate accumulation:
+//   t  = s x A^T        (rows = tokens,   cols = rank; reduction over in-features)
+//   u  = s dY B         (rows = tokens,   cols = rank; reduction over out-features)
+//   dA^T = x^T u        (rows = in-features,  cols = rank; reduction over tokens)
+//   dB   = dY^T t       (rows = out-features, cols = rank; reduction over tokens)
+//
+// "QLoRA Paper Breakdown: 4-Bit NormalFloat (NF4), Double Quantization, and Paged
+// Optimizers" (fullstackaihub), section 4: the adapter term (alpha/r) X L1 L2 of the forward
+// pass and the adapter-only gradients of the backward; "QLoRA, explained." step 5.
+//
+// The tensor cores multiply exact bf16 values (x, dY, A, B, or an exact three-term bf16
+// split of an fp32 t or u: fp32 = t1 + t2 + t3 with 8 significant bits each) and accumulate
+// one 64-wide k-block at a time in TMEM (fp32).  After every k-block the epilogue warps move
+// the block sums into float64 registers (TMEM is double-buffered so the next k-block's MMAs
+// overlap the flush), adding the three split terms of a column in float64.  The float64
+// partial of each K split goes to the workspace; a finalize kernel sums the splits.  With
+// the long reductions here (thousands of tokens), plain fp32 accumulation leaves errors far
+// above the elementwise absolute floor at outputs that cancel to near zero; this keeps the
+// error at the level of one fp32 rounding per 64-wide block.
+#pragma once
+
+#include "nf4_device.cuh"
+
+namespace qnf4 {
+
+struct LowRankParams {
+  CUtensorMap a_map;      // A operand (K-major: rows x k, or MN-major: k x rows)
+  CUtensorMap b_map[3];   // B operand terms, each K-major [cols][k]
+  int32_t a_mn;           // A operand is MN-major (two 64-row boxes per k-block)
+  int32_t kblocks, k16_last;
+  int32_t splits, kb_per_split;
+  int32_t rows, cols;     // valid extent: rows on the UMMA M side, cols = rank columns
+  double* partial;        // [splits][cols][rows] float64
+};
+
+constexpr int kLrThreads = 192;
+
+template <int BJ, int TERMS>
+struct LrCfg {
+  static constexpr int BN = BJ * TERMS;            // UMMA N
+  static constexpr int kABytes = 128 * 64 * 2;
+  static constexpr int kBTermBytes = BJ * 64 * 2;
+  static constexpr int kBBytes = TERMS * kBTermBytes;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kStagesRaw = (200 * 1024) / kStageBytes;
+  static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
+  static constexpr int kTmemCols = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
+                                   : (2 * BN <= 256) ? 256 : 512;
+  static constexpr int kSmemBytes = kStages * kStageBytes + 256 + 1024;
+  static_assert(BN % 16 == 0 && BN <= 256, "UMMA N");
+  static_assert(kBTermBytes % 1024 == 0, "term boxes keep the swizzle atom alignment");
+};
+
+__device__ __forceinline__ void tmem_ld_32x32b_x16_lr(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
+template <int BJ, int TERMS>
+__global__ void __launch_bounds__(kLrThreads, 1) lowrank_kernel(const __grid_constant__ LowRankParams p) {
+  using C = LrCfg<BJ, TERMS>;
+  constexpr int S = C::kStages;
+  extern __shared__ uint8_t smem_dyn[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
+  uint64_t* empty = full + S;
+  uint64_t* accfull = empty + S;      // [2]
+  uint64_t* accempty = accfull + 2;   // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accempty + 2);
+  volatile uint32_t* abort_word = tmem_slot + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row0 = blockIdx.x * 128, col0 = blockIdx.y * BJ, split = blockIdx.z;
+  const int kb_begin = split * p.kb_per_split;
+  int kb_end = kb_begin + p.kb_per_split;
+  if (kb_end > p.kblocks) kb_end = p.kblocks;
+  const int n_iters = kb_end > kb_begin ? kb_end - kb_begin : 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&accfull[b], 1);
+      mbar_init(&accempty[b], 4);
+    }
+    *abort_word = 0u;
+    mbar_fence_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&p.a_map);
+    for (int t = 0; t < TERMS; ++t) tma_prefetch_desc(&p.b_map[t]);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA
+    int last_issue[8];
+    for (int s = 0; s < 8; ++s) last_issue[s] = -1;
+    bool ok = true;
+    for (int it = 0; it < n_iters; ++it) {
+      const int s = it % S;
+      const uint32_t ph = (uint32_t)(it / S) & 1u;
+      if (!mbar_wait(&empty[s], ph ^ 1u, abort_word, kErrWaitEmpty)) { ok = false; break; }
+      if (lane == 0) {
+        uint8_t* A = smem + s * C::kStageBytes;
+        uint8_t* B = A + C::kABytes;
+        mbar_arrive_expect_tx(&full[s], C::kABytes + C::kBBytes);
+        const int k = (kb_begin + it) * 64;
+        if (p.a_mn) {
+          tma_load_2d(A, &p.a_map, row0, k, &full[s]);
+          tma_load_2d(A + 8192, &p.a_map, row0 + 64, k, &full[s]);
+        } else {
+          tma_load_2d(A, &p.a_map, k, row0, &full[s]);
+        }
+#pragma unroll
+        for (int t = 0; t < TERMS; ++t) tma_load_2d(B + t * C::kBTermBytes, &p.b_map[t], k, col0, &full[s]);
+        last_issue[s] = it;
+      }
+      __syncwarp();
+    }
+    if (!ok && lane == 0) {
+      for (int s = 0; s < S; ++s)
+        if (last_issue[s] >= 0) {
+          const uint32_t ph = (uint32_t)(last_issue[s] / S) & 1u;
+          for (int i = 0; i < (1 << 20) && !mbar_try_wait(&full[s], ph); ++i) {}
+        }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA
+    const uint32_t idesc = umma_idesc_bf16(128, C::BN, p.a_mn ? 1u : 0u, 0u);
+    for (int it = 0; it < n_iters; ++it) {
+      const int s = it % S;
+      const uint32_t ph = (uint32_t)(it / S) & 1u;
+      const int buf = it & 1;
+      const uint32_t bph = (uint32_t)(it >> 1) & 1u;
+      if (!mbar_wait(&accempty[buf], bph ^ 1u, abort_word, kErrWaitMma)) break;
+      if (!mbar_wait(&full[s], ph, abort_word, kErrWaitTma)) break;
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t a_addr = smem_u32(smem + s * C::kStageBytes);
+        const uint32_t b_addr = a_addr + C::kABytes;
+        const int nk16 = (kb_begin + it == p.kblocks - 1) ? p.k16_last : 4;
+        const uint32_t d = tmem_base + (uint32_t)(buf * C::BN);
+        for (int k16 = 0; k16 < nk16; ++k16) {
+          const uint64_t ad = p.a_mn ? umma_sdesc_sw128(a_addr + (uint32_t)k16 * 2048u, 8192u, 1024u)
+                                     : umma_sdesc_sw128(a_addr + (uint32_t)k16 * 32u, 16u, 1024u);
+          const uint64_t bd = umma_sdesc_sw128(b_addr + (uint32_t)k16 * 32u, 16u, 1024u);
+          umma_bf16(d, ad, bd, idesc, k16 > 0 ? 1u : 0u);
+        }
+        umma_commit(&empty[s]);
+        umma_commit(&accfull[buf]);
+      }
+      __syncwarp();
+    }
+  } else {
+    // ------------------------------------------------------------------ flush to float64
+    const int q = warp & 3;
+    const int row = row0 + 32 * q + lane;
+    double acc[BJ];
+#pragma unroll
+    for (int j = 0; j < BJ; ++j) acc[j] = 0.0;
+    bool ok = true;
+    for (int it = 0; it < n_iters; ++it) {
+      const int buf = it & 1;
+      const uint32_t bph = (uint32_t)(it >> 1) & 1u;
+      if (!mbar_wait(&accfull[buf], bph, abort_word, kErrWaitMma)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t tb = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * C::BN);
+#pragma unroll
+      for (int j0 = 0; j0 < BJ; j0 += 16) {
+        uint32_t r[TERMS][16];
+#pragma unroll
+        for (int t = 0; t < TERMS; ++t) tmem_ld_32x32b_x16_lr(tb + (uint32_t)(t * BJ + j0), r[t]);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          double v = (double)__uint_as_float(r[0][j]);
+#pragma unroll
+          for (int t = 1; t < TERMS; ++t) v += (double)__uint_as_float(r[t][j]);
+          acc[j0 + j] += v;
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&accempty[buf]);
+    }
+    if (ok && row < p.rows) {
+      double* out = p.partial + (int64_t)split * p.cols * p.rows;
+#pragma unroll
+      for (int j = 0; j < BJ; ++j) {
+        const int col = col0 + j;
+        if (col < p.cols) out[(int64_t)col * p.rows + row] = acc[j];
+      }
+    }
+    tc_fence_before();
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+template <int BJ, int TERMS>
+static cudaError_t launch_lowrank_t(const LowRankParams& p, cudaStream_t st) {
+  using C = LrCfg<BJ, TERMS>;
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(lowrank_kernel<BJ, TERMS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  dim3 grid((p.rows + 127) / 128, (p.cols + BJ - 1) / BJ, p.splits);
+  lowrank_kernel<BJ, TERMS><<<grid, kLrThreads, C::kSmemBytes, st>>>(p);
+  return cudaGetLastError();
+}
+
+// bj in {16, 32, 64}, terms in {1, 3}
+static cudaError_t launch_lowrank(const LowRankParams& p, int bj, int terms, cudaStream_t st) {
+  if (terms == 1) {
+    if (bj == 16) return launch_lowrank_t<16, 1>(p, st);
+    if (bj == 32) return launch_lowrank_t<32, 1>(p, st);
+    if (bj == 64) return launch_lowrank_t<64, 1>(p, st);
+  } else if (terms == 3) {
+    if (bj == 16) return launch_lowrank_t<16, 3>(p, st);
+    if (bj == 32) return launch_lowrank_t<32, 3>(p, st);
+    if (bj == 64) return launch_lowrank_t<64, 3>(p, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+// ---------------------------------------------------------------------------------------
+// finalize kernels
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ uint16_t bf16_bits_rn(double v) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn((float)v));
+}
+
+// Three bf16 terms of v: t1 = bf16(v), t2 = bf16(v - t1), t3 = bf16(v - t1 - t2), each
+// difference formed in float64.  For an fp32 v the three terms are exact (8 + 8 + 8 bits).
+__device__ __forceinline__ void split3(double v, uint16_t& a, uint16_t& b, uint16_t& c) {
+  const __nv_bfloat16 h1 = __float2bfloat16_rn((float)v);
+  const double r1 = v - (double)__bfloat162float(h1);
+  const __nv_bfloat16 h2 = __float2bfloat16_rn((float)r1);
+  const double r2 = r1 - (double)__bfloat162float(h2);
+  a = __bfloat16_as_ushort(h1);
+  b = __bfloat16_as_ushort(h2);
+  c = __bfloat16_as_ushort(__float2bfloat16_rn((float)r2));
+}
+
+// Token-side result (t or u): v = alpha * sum_z partial[z][j][m].  Optional outputs:
+// fp32 [M][r]; bf16 hi / lo [M][r] (two-term split, for the fused GEMMs' adapter k-blocks);
+// the three-term split transposed, T3[term][j][m] with row pitch ldT (for dA / dB).
+__global__ void finalize_tokens_kernel(const double* __restrict__ partial, int splits, int64_t M, int64_t r,
+                                       double alpha, float* __restrict__ f32, uint16_t* __restrict__ hi,
+                                       uint16_t* __restrict__ lo, uint16_t* __restrict__ T3, int64_t ldT) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= M * r) return;
+  const int64_t j = idx / M, m = idx % M;
+  double v = 0.0;
+  for (int z = 0; z < splits; ++z) v += partial[((int64_t)z * r + j) * M + m];
+  v *= alpha;
+  if (f32) f32[m * r + j] = (float)v;
+  if (hi) {
+    const __nv_bfloat16 h = __float2bfloat16_rn((float)v);
+    hi[m * r + j] = __bfloat16_as_ushort(h);
+    lo[m * r + j] = bf16_bits_rn(v - (double)__bfloat162float(h));
+  }
+  if (T3) {
+    uint16_t a, b, c;
+    split3(v, a, b, c);
+    T3[j * ldT + m] = a;
+    T3[(r + j) * ldT + m] = b;
+    T3[(2 * r + j) * ldT + m] = c;
+  }
+}
+
+// fp32 t [M][r] -> exact three-term split, transposed: T3[term][j][m].
+__global__ void split3_T_kernel(const float* __restrict__ t, int64_t M, int64_t r, uint16_t* __restrict__ T3,
+                                int64_t ldT) {
+  __shared__ float tile[32][33];
+  const int64_t m0 = (int64_t)blockIdx.y * 32, j0 = (int64_t)blockIdx.x * 32;
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int64_t m = m0 + i, j = j0 + threadIdx.x;
+    tile[i][threadIdx.x] = (m < M && j < r) ? t[m * r + j] : 0.0f;
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int64_t j = j0 + i, m = m0 + threadIdx.x;
+    if (m < M && j < r) {
+      uint16_t a, b, c;
+      split3((double)tile[threadIdx.x][i], a, b, c);
+      T3[j * ldT + m] = a;
+      T3[(r + j) * ldT + m] = b;
+      T3[(2 * r + j) * ldT + m] = c;
+    }
+  }
+}
+
+// Feature-side gradient: g[j][i] = bf16(sum_z partial[z][j][i]); transpose_out = 0 writes
+// out[j * n + i] (dA, [r][K]), 1 writes out[i * r + j] (dB, [N][r]).
+__global__ void finalize_grad_kernel(const double* __restrict__ partial, int splits, int64_t r, int64_t n,
+                                     uint16_t* __restrict__ out, int transpose_out) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= r * n) return;
+  int64_t j, i;
+  if (transpose_out) { i = idx / r; j = idx % r; }
+  else { j = idx / n; i = idx % n; }
+  double v = 0.0;
+  for (int z = 0; z < splits; ++z) v += partial[((int64_t)z * r + j) * n + i];
+  out[idx] = bf16_bits_rn(v);
+}
+
+static cudaError_t launch_finalize_tokens(const double* partial, int splits, int64_t M, int64_t r, double alpha,
+                                          float* f32, uint16_t* hi, uint16_t* lo, uint16_t* T3, int64_t ldT,
+                                          cudaStream_t st) {
+  const int64_t n = M * r;
+  finalize_tokens_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(partial, splits, M, r, alpha, f32, hi, lo,
+                                                                       T3, ldT);
+  return cudaGetLastError();
+}
+
+static cudaError_t launch_split3_T(const float* t, int64_t M, int64_t r, uint16_t* T3, int64_t ldT,
+                                   cudaStream_t st) {
+  dim3 grid((unsigned)((r + 31) / 32), (unsigned)((M + 31) / 32));
+  split3_T_kernel<<<grid, dim3(32, 8), 0, st>>>(t, M, r, T3, ldT);
+  return cudaGetLastError();
+}
+
+static cudaError_t launch_finalize_grad(const double* partial, int splits, int64_t r, int64_t n, uint16_t* out,
+                                        int transpose_out, cudaStream_t st) {
+  const int64_t total = r * n;
+  finalize_grad_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(partial, splits, r, n, out, transpose_out);
+  return cudaGetLastError();
+}
+
+}  // namespace qnf4

@@ -2,12 +2,14 @@
 // (argument checks, workspace layout, TMA tensor maps, kernel sequencing).
 #include <cstdarg>
 #include <cstdio>
+#include <algorithm>
 #include <cstring>
 #include <string>
 
 #include "qlora_nf4.h"
 #include "codec.cuh"
 #include "gemm.cuh"
+#include "lowrank.cuh"
 
 namespace {
 
@@ -150,9 +152,24 @@ struct Carver {
   }
 };
 
+// Column tile of the low-rank kernels (rank columns per CTA).
+int bj_for(int r) { return r <= 16 ? 16 : (r <= 32 ? 32 : 64); }
+
+struct LowRankPlan {
+  int bj, splits;
+};
+
+LowRankPlan plan_lowrank(int64_t rows, int r, int64_t kdim) {
+  LowRankPlan p;
+  p.bj = bj_for(r);
+  const int64_t tiles = ((rows + 127) / 128) * ((r + p.bj - 1) / p.bj);
+  p.splits = choose_splits(tiles, kblocks(kdim));
+  return p;
+}
+
 struct FwdPlan {
-  int bn, splits;
-  int bn_t;
+  int bn, splits;   // fused forward
+  LowRankPlan t;    // t = s x A^T
 };
 
 FwdPlan plan_fwd(const LinearShape& s) {
@@ -160,14 +177,13 @@ FwdPlan plan_fwd(const LinearShape& s) {
   p.bn = bn_for(s.M);
   const int64_t tiles = ((s.N + 127) / 128) * ((s.M + p.bn - 1) / p.bn);
   p.splits = choose_splits(tiles, kblocks(s.K));
-  p.bn_t = bn_for(s.r);
+  p.t = plan_lowrank(s.M, s.r, s.K);
   return p;
 }
 
 struct BwdPlan {
-  int bn, splits;         // dX
-  int bn_u;               // u = s dY B
-  int bn_g, splits_a, splits_b;   // dA / dB
+  int bn, splits;      // fused dX
+  LowRankPlan u, a, b; // u = s dY B, dA, dB
 };
 
 BwdPlan plan_bwd(const LinearShape& s) {
@@ -175,24 +191,30 @@ BwdPlan plan_bwd(const LinearShape& s) {
   p.bn = bn_for(s.M);
   const int64_t tiles = ((s.K + 127) / 128) * ((s.M + p.bn - 1) / p.bn);
   p.splits = choose_splits(tiles, kblocks(s.N));
-  p.bn_u = bn_for(s.r);
-  p.bn_g = bn_for(2 * s.r);
-  const int64_t cg = (2 * s.r + p.bn_g - 1) / p.bn_g;
-  p.splits_a = choose_splits(((s.K + 127) / 128) * cg, kblocks(s.M));
-  p.splits_b = choose_splits(((s.N + 127) / 128) * cg, kblocks(s.M));
+  p.u = plan_lowrank(s.M, s.r, s.N);
+  p.a = plan_lowrank(s.K, s.r, s.M);
+  p.b = plan_lowrank(s.N, s.r, s.M);
   return p;
 }
 
-size_t fwd_carve(Carver& c, const LinearShape& s, const FwdPlan& p, uint16_t** thi, uint16_t** tlo, float** part) {
-  *thi = c.take<uint16_t>((size_t)s.M * s.r);
-  *tlo = c.take<uint16_t>((size_t)s.M * s.r);
-  *part = p.splits > 1 ? c.take<float>((size_t)p.splits * s.M * s.N) : nullptr;
+struct FwdWs {
+  uint16_t *thi, *tlo;
+  double* partial;
+  float* part;
+};
+
+size_t fwd_carve(Carver& c, const LinearShape& s, const FwdPlan& p, FwdWs* w) {
+  w->thi = c.take<uint16_t>((size_t)s.M * s.r);
+  w->tlo = c.take<uint16_t>((size_t)s.M * s.r);
+  w->partial = c.take<double>((size_t)p.t.splits * s.r * s.M);
+  w->part = p.splits > 1 ? c.take<float>((size_t)p.splits * s.M * s.N) : nullptr;
   return c.off;
 }
 
 struct BwdWs {
-  uint16_t *Bt, *uhi, *ulo, *uT, *tT;
-  float *partX, *partA, *partB;
+  uint16_t *Bt, *uhi, *ulo, *uT3, *tT3;
+  double* partial;
+  float* partX;
 };
 
 size_t bwd_carve(Carver& c, const LinearShape& s, const BwdPlan& p, BwdWs* w) {
@@ -200,12 +222,41 @@ size_t bwd_carve(Carver& c, const LinearShape& s, const BwdPlan& p, BwdWs* w) {
   w->Bt = c.take<uint16_t>((size_t)s.r * s.N);
   w->uhi = c.take<uint16_t>((size_t)s.M * s.r);
   w->ulo = c.take<uint16_t>((size_t)s.M * s.r);
-  w->uT = c.take<uint16_t>((size_t)2 * s.r * ldM);
-  w->tT = c.take<uint16_t>((size_t)2 * s.r * ldM);
+  w->uT3 = c.take<uint16_t>((size_t)3 * s.r * ldM);
+  w->tT3 = c.take<uint16_t>((size_t)3 * s.r * ldM);
+  size_t np = (size_t)p.u.splits * s.r * s.M;
+  np = std::max(np, (size_t)p.a.splits * s.r * s.K);
+  np = std::max(np, (size_t)p.b.splits * s.r * s.N);
+  w->partial = c.take<double>(np);
   w->partX = p.splits > 1 ? c.take<float>((size_t)p.splits * s.M * s.K) : nullptr;
-  w->partA = c.take<float>((size_t)p.splits_a * 2 * s.r * s.K);
-  w->partB = c.take<float>((size_t)p.splits_b * 2 * s.r * s.N);
   return c.off;
+}
+
+// One low-rank product: A operand map (K-major over [rows][k] or MN-major over [k][rows]),
+// `terms` B maps over [r][k] (K-major), fp64 partials into `partial`.
+int run_lowrank(const void* a_base, bool a_mn, int64_t a_inner, int64_t a_outer, int64_t a_pitch_bytes,
+                const uint16_t* const* b_terms, int terms, int64_t b_inner, int64_t b_pitch_bytes, int r,
+                int64_t rows, int64_t kdim, const LowRankPlan& pl, double* partial, cudaStream_t st) {
+  qnf4::LowRankParams lp;
+  memset(&lp, 0, sizeof(lp));
+  if (a_mn) {
+    if (int rc = make_map(&lp.a_map, a_base, true, a_inner, a_outer, a_pitch_bytes, 64, 64)) return rc;
+  } else {
+    if (int rc = make_map(&lp.a_map, a_base, true, a_inner, a_outer, a_pitch_bytes, 64, 128)) return rc;
+  }
+  for (int t = 0; t < terms; ++t)
+    if (int rc = make_map(&lp.b_map[t], b_terms[t], true, b_inner, r, b_pitch_bytes, 64, pl.bj)) return rc;
+  lp.a_mn = a_mn ? 1 : 0;
+  lp.kblocks = kblocks(kdim);
+  lp.k16_last = k16_last(kdim);
+  lp.splits = pl.splits;
+  lp.kb_per_split = (lp.kblocks + pl.splits - 1) / pl.splits;
+  lp.rows = (int32_t)rows;
+  lp.cols = r;
+  lp.partial = partial;
+  cudaError_t e = qnf4::launch_lowrank(lp, pl.bj, terms, st);
+  if (e != cudaSuccess) return cuda_fail(e, "low-rank launch");
+  return QNF4_OK;
 }
 
 int nf4_operand(qnf4::GemmParams& gp, const uint8_t* codes, const uint8_t* scale_codes, const float* c2,
@@ -297,9 +348,8 @@ size_t qlora_linear_fwd_workspace_bytes(int64_t M, int64_t K, int64_t N, int r) 
   LinearShape s{M, K, N, r};
   if (M <= 0 || K <= 0 || N <= 0 || r <= 0) return 0;
   Carver c{nullptr};
-  uint16_t *a, *b;
-  float* p;
-  return fwd_carve(c, s, plan_fwd(s), &a, &b, &p);
+  FwdWs w;
+  return fwd_carve(c, s, plan_fwd(s), &w);
 }
 
 int qlora_linear_fwd(const uint16_t* x, int64_t M, int64_t K, int64_t N, const uint8_t* codes,
@@ -316,35 +366,20 @@ int qlora_linear_fwd(const uint16_t* x, int64_t M, int64_t K, int64_t N, const u
     return fail(QNF4_ERR_UNSUPPORTED, "alignment: operands 16 B, workspace 256 B");
   const FwdPlan plan = plan_fwd(sh);
   Carver c{static_cast<char*>(workspace)};
-  uint16_t *thi, *tlo;
-  float* part;
-  const size_t need = fwd_carve(c, sh, plan, &thi, &tlo, &part);
+  FwdWs w;
+  const size_t need = fwd_carve(c, sh, plan, &w);
   if (workspace_bytes < need) return fail(QNF4_ERR_WORKSPACE, "workspace needs %zu bytes", need);
   if (int rc = check_arch()) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   mark(0, st);
 
-  // 1) t = s x A^T (fp32 to t_saved), hi / lo bf16 parts to the workspace
+  // 1) t = s x A^T: float64-accumulated partials, then t (fp32) and its bf16 hi / lo parts
   {
-    qnf4::GemmParams gp;
-    memset(&gp, 0, sizeof(gp));
-    if (int rc = make_map(&gp.maps[0], x, true, K, M, K * 2, 64, 128)) return rc;
-    if (int rc = make_map(&gp.maps[1], A, true, K, r, K * 2, 64, plan.bn_t)) return rc;
-    gp.nseg = 1;
-    gp.seg[0] = qnf4::GemmSeg{kblocks(K), k16_last(K), qnf4::kATmaK, 0, 1, 0, 0, 0};
-    gp.rows = (int32_t)M;
-    gp.cols = r;
-    gp.splits = 1;
-    gp.kb_per_split = kblocks(K);
-    gp.epi = qnf4::kEpiRowHiLo;
-    gp.alpha = s;
-    gp.out = t_saved;
-    gp.ld_out = r;
-    gp.hi = thi;
-    gp.lo = tlo;
-    gp.ld_hl = r;
-    cudaError_t e = qnf4::launch_gemm(gp, plan.bn_t, st);
-    if (e != cudaSuccess) return cuda_fail(e, "down-projection launch");
+    const uint16_t* bt[1] = {A};
+    if (int rc = run_lowrank(x, false, K, M, K * 2, bt, 1, K, K * 2, r, M, K, plan.t, w.partial, st)) return rc;
+    cudaError_t e = qnf4::launch_finalize_tokens(w.partial, plan.t.splits, M, r, (double)s, t_saved, w.thi, w.tlo,
+                                                 nullptr, 0, st);
+    if (e != cudaSuccess) return cuda_fail(e, "finalize launch");
   }
   mark(1, st);
   // 2) y^T = W' x^T + B t_hi^T + B t_lo^T, W' dequantized on chip
@@ -357,8 +392,8 @@ int qlora_linear_fwd(const uint16_t* x, int64_t M, int64_t K, int64_t N, const u
     }
     if (int rc = make_map(&gp.maps[1], x, true, K, M, K * 2, 64, plan.bn)) return rc;
     if (int rc = make_map(&gp.maps[2], B, true, r, N, (uint64_t)r * 2, 64, 128)) return rc;
-    if (int rc = make_map(&gp.maps[3], thi, true, r, M, (uint64_t)r * 2, 64, plan.bn)) return rc;
-    if (int rc = make_map(&gp.maps[4], tlo, true, r, M, (uint64_t)r * 2, 64, plan.bn)) return rc;
+    if (int rc = make_map(&gp.maps[3], w.thi, true, r, M, (uint64_t)r * 2, 64, plan.bn)) return rc;
+    if (int rc = make_map(&gp.maps[4], w.tlo, true, r, M, (uint64_t)r * 2, 64, plan.bn)) return rc;
     nf4_operand(gp, codes, scale_codes, c2, mean, N, K);
     gp.nseg = 3;
     gp.seg[0] = qnf4::GemmSeg{kblocks(K), k16_last(K), qnf4::kANf4K, 0, 1, 0, 0, 0};
@@ -370,7 +405,7 @@ int qlora_linear_fwd(const uint16_t* x, int64_t M, int64_t K, int64_t N, const u
     gp.kb_per_split = (kblocks(K) + plan.splits - 1) / plan.splits;
     if (plan.splits > 1) {
       gp.epi = qnf4::kEpiF32T;
-      gp.out = part;
+      gp.out = w.part;
       gp.ld_out = N;
       gp.split_stride = M * N;
     } else {
@@ -381,7 +416,7 @@ int qlora_linear_fwd(const uint16_t* x, int64_t M, int64_t K, int64_t N, const u
     cudaError_t e = qnf4::launch_gemm(gp, plan.bn, st);
     if (e != cudaSuccess) return cuda_fail(e, "fused forward launch");
     if (plan.splits > 1) {
-      e = qnf4::launch_reduce_splits_bf16(part, plan.splits, M * N, M, N, N, y, N, st);
+      e = qnf4::launch_reduce_splits_bf16(w.part, plan.splits, M * N, M, N, N, y, N, st);
       if (e != cudaSuccess) return cuda_fail(e, "split reduce launch");
     }
   }
@@ -396,8 +431,10 @@ int qlora_linear_plan(int64_t M, int64_t K, int64_t N, int r, int* fwd_launches,
   if (int rc = check_linear_shape(sh)) return rc;
   const FwdPlan f = plan_fwd(sh);
   const BwdPlan b = plan_bwd(sh);
-  if (fwd_launches) *fwd_launches = 2 + (f.splits > 1 ? 1 : 0);
-  if (bwd_launches) *bwd_launches = 8 + (b.splits > 1 ? 1 : 0);
+  // forward: t, finalize, fused (+ split reduce); backward: B^T, t split, u, finalize,
+  // fused dX (+ split reduce), dA, finalize, dB, finalize
+  if (fwd_launches) *fwd_launches = 3 + (f.splits > 1 ? 1 : 0);
+  if (bwd_launches) *bwd_launches = 9 + (b.splits > 1 ? 1 : 0);
   if (fwd_splits) *fwd_splits = f.splits;
   if (dx_splits) *dx_splits = b.splits;
   return QNF4_OK;
@@ -435,36 +472,20 @@ int qlora_linear_bwd(const uint16_t* dY, const uint16_t* x, const float* t_saved
   cudaError_t e;
   mark(0, st);
 
-  // 1) B^T [r][N] and t split into transposed hi / lo rows [2r][M]
+  // 1) B^T [r][N]; t split into three exact bf16 terms, transposed [3][r][M]
   e = qnf4::launch_transpose_bf16(B, N, r, w.Bt, N, st);
   if (e != cudaSuccess) return cuda_fail(e, "transpose launch");
-  e = qnf4::launch_split_hilo_T(t_saved, M, r, w.tT, ldM, st);
+  e = qnf4::launch_split3_T(t_saved, M, r, w.tT3, ldM, st);
   if (e != cudaSuccess) return cuda_fail(e, "split launch");
   mark(1, st);
 
-  // 2) u = s dY B: hi / lo as [M][r] (dX adapter operand) and as [2r][M] (dA operand)
+  // 2) u = s dY B (float64-accumulated): hi / lo [M][r] for dX, three terms [3][r][M] for dA
   {
-    qnf4::GemmParams gp;
-    memset(&gp, 0, sizeof(gp));
-    if (int rc = make_map(&gp.maps[0], dY, true, N, M, N * 2, 64, 128)) return rc;
-    if (int rc = make_map(&gp.maps[1], w.Bt, true, N, r, N * 2, 64, plan.bn_u)) return rc;
-    gp.nseg = 1;
-    gp.seg[0] = qnf4::GemmSeg{kblocks(N), k16_last(N), qnf4::kATmaK, 0, 1, 0, 0, 0};
-    gp.rows = (int32_t)M;
-    gp.cols = r;
-    gp.splits = 1;
-    gp.kb_per_split = kblocks(N);
-    gp.epi = qnf4::kEpiRowHiLo;
-    gp.alpha = s;
-    gp.out = nullptr;
-    gp.hi = w.uhi;
-    gp.lo = w.ulo;
-    gp.ld_hl = r;
-    gp.hiT = w.uT;
-    gp.loT = w.uT + (size_t)r * ldM;
-    gp.ld_T = ldM;
-    e = qnf4::launch_gemm(gp, plan.bn_u, st);
-    if (e != cudaSuccess) return cuda_fail(e, "up-projection launch");
+    const uint16_t* bt[1] = {w.Bt};
+    if (int rc = run_lowrank(dY, false, N, M, N * 2, bt, 1, N, N * 2, r, M, N, plan.u, w.partial, st)) return rc;
+    e = qnf4::launch_finalize_tokens(w.partial, plan.u.splits, M, r, (double)s, nullptr, w.uhi, w.ulo, w.uT3, ldM,
+                                     st);
+    if (e != cudaSuccess) return cuda_fail(e, "finalize launch");
   }
   mark(2, st);
   // 3) dX^T = W'^T dY^T + A^T u_hi^T + A^T u_lo^T
@@ -506,48 +527,20 @@ int qlora_linear_bwd(const uint16_t* dY, const uint16_t* x, const float* t_saved
     }
   }
   mark(3, st);
-  // 4) dA^T = x^T [u_hi | u_lo]   (rows K, cols 2r, reduced over M)
+  // 4) dA^T = x^T u (u as three terms), reduced over the M tokens
   {
-    qnf4::GemmParams gp;
-    memset(&gp, 0, sizeof(gp));
-    if (int rc = make_map(&gp.maps[0], x, true, K, M, K * 2, 64, 64)) return rc;
-    if (int rc = make_map(&gp.maps[1], w.uT, true, M, 2 * r, ldM * 2, 64, plan.bn_g)) return rc;
-    gp.nseg = 1;
-    gp.seg[0] = qnf4::GemmSeg{kblocks(M), k16_last(M), qnf4::kATmaMN, 0, 1, 0, 0, 0};
-    gp.rows = (int32_t)K;
-    gp.cols = 2 * r;
-    gp.splits = plan.splits_a;
-    gp.kb_per_split = (kblocks(M) + plan.splits_a - 1) / plan.splits_a;
-    gp.epi = qnf4::kEpiF32T;
-    gp.out = w.partA;
-    gp.ld_out = K;
-    gp.split_stride = 2 * r * K;
-    e = qnf4::launch_gemm(gp, plan.bn_g, st);
-    if (e != cudaSuccess) return cuda_fail(e, "dA launch");
-    e = qnf4::launch_reduce_hilo(w.partA, plan.splits_a, 2 * r * K, r, K, K, dA, 0, st);
-    if (e != cudaSuccess) return cuda_fail(e, "dA reduce launch");
+    const uint16_t* bt[3] = {w.uT3, w.uT3 + (size_t)r * ldM, w.uT3 + (size_t)2 * r * ldM};
+    if (int rc = run_lowrank(x, true, K, M, K * 2, bt, 3, M, ldM * 2, r, K, M, plan.a, w.partial, st)) return rc;
+    e = qnf4::launch_finalize_grad(w.partial, plan.a.splits, r, K, dA, 0, st);
+    if (e != cudaSuccess) return cuda_fail(e, "dA finalize launch");
   }
   mark(4, st);
-  // 5) dB = dY^T [t_hi | t_lo]   (rows N, cols 2r, reduced over M)
+  // 5) dB = dY^T t (t as three terms), reduced over the M tokens
   {
-    qnf4::GemmParams gp;
-    memset(&gp, 0, sizeof(gp));
-    if (int rc = make_map(&gp.maps[0], dY, true, N, M, N * 2, 64, 64)) return rc;
-    if (int rc = make_map(&gp.maps[1], w.tT, true, M, 2 * r, ldM * 2, 64, plan.bn_g)) return rc;
-    gp.nseg = 1;
-    gp.seg[0] = qnf4::GemmSeg{kblocks(M), k16_last(M), qnf4::kATmaMN, 0, 1, 0, 0, 0};
-    gp.rows = (int32_t)N;
-    gp.cols = 2 * r;
-    gp.splits = plan.splits_b;
-    gp.kb_per_split = (kblocks(M) + plan.splits_b - 1) / plan.splits_b;
-    gp.epi = qnf4::kEpiF32T;
-    gp.out = w.partB;
-    gp.ld_out = N;
-    gp.split_stride = 2 * r * N;
-    e = qnf4::launch_gemm(gp, plan.bn_g, st);
-    if (e != cudaSuccess) return cuda_fail(e, "dB launch");
-    e = qnf4::launch_reduce_hilo(w.partB, plan.splits_b, 2 * r * N, r, N, N, dB, 1, st);
-    if (e != cudaSuccess) return cuda_fail(e, "dB reduce launch");
+    const uint16_t* bt[3] = {w.tT3, w.tT3 + (size_t)r * ldM, w.tT3 + (size_t)2 * r * ldM};
+    if (int rc = run_lowrank(dY, true, N, M, N * 2, bt, 3, M, ldM * 2, r, N, M, plan.b, w.partial, st)) return rc;
+    e = qnf4::launch_finalize_grad(w.partial, plan.b.splits, r, N, dB, 1, st);
+    if (e != cudaSuccess) return cuda_fail(e, "dB finalize launch");
   }
   mark(5, st);
   return QNF4_OK;

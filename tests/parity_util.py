@@ -39,13 +39,24 @@ def assert_within_tolerance(got: torch.Tensor | np.ndarray, ref: np.ndarray, wha
     assert fro <= FRO_TOL, f"{what}: relative Frobenius error {fro:.3e}"
 
 
+_WEIGHT_CACHE: dict = {}
+
+
 def oracle_weight(w_bf16: torch.Tensor) -> dict:
-    """Oracle quantize + dequant of a bf16 weight; W' as float64 [N][K] plus the codec parts."""
+    """Oracle quantize + dequant of a bf16 weight; W' as float64 [N][K] plus the codec parts
+    (memoised on the weight's bytes: several tests share one weight)."""
+    import hashlib
+    key = (tuple(w_bf16.shape), hashlib.sha1(w_bf16.contiguous().view(torch.int16).numpy().tobytes()).hexdigest())
+    if key in _WEIGHT_CACHE:
+        return _WEIGHT_CACHE[key]
     w = w_bf16.float().cpu().numpy().ravel()
     qd = onf4.quantize_nf4_dq(w)
     bits = onf4.dequant_nf4_dq(qd["codes"], qd["scale_codes"], qd["c2"], qd["mean"], w.size)
     qd["w_deq_bits"] = bits
     qd["w_deq"] = onf4.bf16_bits_to_f32(bits).astype(np.float64).reshape(tuple(w_bf16.shape))
+    if len(_WEIGHT_CACHE) > 4:
+        _WEIGHT_CACHE.clear()
+    _WEIGHT_CACHE[key] = qd
     return qd
 
 
