@@ -24,8 +24,14 @@ enum : uint32_t {
 // library is compiled as a single translation unit, so the definition lives here.
 __device__ uint32_t g_error_word = 0;
 
-// Roughly seconds of spinning before a wait gives up (each try_wait may itself suspend).
-constexpr uint32_t kWaitLimit = 1u << 26;
+// A bounded wait gives up after this much wall-clock time (%globaltimer, nanoseconds).
+constexpr uint64_t kWaitLimitNs = 4000000000ull;
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -58,14 +64,32 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// try_wait that may suspend the thread for up to `hint_ns` while the phase is incomplete
+// (the thread resumes as soon as the phase completes).
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
 // Bounded wait: returns false (and raises `flag` in the device error word and in the
-// CTA-local abort word) if the phase did not complete within kWaitLimit tries, or if
-// another role of the CTA has already aborted.
+// CTA-local abort word) if the phase did not complete within kWaitLimitNs of wall-clock
+// time, or if another role of the CTA has already aborted.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile uint32_t* abort_word,
                                           uint32_t flag) {
-  for (uint32_t i = 0; i < kWaitLimit; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 1023u) == 1023u && *abort_word) return false;
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait_sleep(bar, parity, 1000u)) return true;
+    if ((i & 15u) == 0u) {
+      if (*abort_word) return false;
+      if (global_timer_ns() - t0 > kWaitLimitNs) break;
+    }
   }
   *abort_word = 1u;
   atomicOr(&g_error_word, flag);

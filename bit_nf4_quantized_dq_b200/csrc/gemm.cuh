@@ -15,8 +15,9 @@
 // with the fp32 intermediates t and u split into bf16 hi + lo parts so that the adapter
 // terms keep close to fp32 accuracy through bf16 tensor-core inputs.
 //
-// Warp roles (192 threads): warp 0 issues TMA loads, warp 1 allocates TMEM and issues MMAs,
-// warps 2-5 run the dequant producer and then the epilogue.
+// Warp roles (320 threads): warp 0 issues TMA loads, warp 1 allocates TMEM and issues MMAs,
+// warps 2-9 run the dequant producer (two groups of four warps on alternate k-blocks) and
+// then the epilogue (each group drains half of the accumulator columns).
 #pragma once
 
 #include "nf4_device.cuh"
@@ -26,7 +27,7 @@ namespace qnf4 {
 
 constexpr int kBM = 128;
 constexpr int kBK = 64;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;   // TMA warp, MMA warp, two groups of four producer / epilogue warps
 constexpr int kCodesBytes = 4096;   // packed codes of one 128 x 64 weight tile
 
 template <int BN>
@@ -88,16 +89,16 @@ struct UnitGeom {
   uint32_t swz;   // row & 7
 };
 
-__device__ __forceinline__ UnitGeom unit_geom(int a_src, int t, int row0, int64_t n_base) {
+__device__ __forceinline__ UnitGeom unit_geom(int a_src, int t, int row0, int64_t k) {
   UnitGeom u;
-  if (a_src == kANf4K) {
+  if (a_src == kANf4K) {            // forward: rows of W, k-block k of its columns
     u.n = row0 + t;
-    u.kcol = n_base;                 // for the forward, n_base carries the unit's first column
+    u.kcol = k;
     u.dst = (uint32_t)t * 128u;
     u.swz = (uint32_t)t & 7u;
-  } else {
+  } else {                          // dX: columns row0.. of W, k-block k of its rows
     const int nl = t >> 1, half = t & 1;
-    u.n = n_base + nl;
+    u.n = k + nl;
     u.kcol = (int64_t)row0 + 64 * half;
     u.dst = (uint32_t)half * 8192u + (uint32_t)nl * 128u;
     u.swz = (uint32_t)nl & 7u;
@@ -105,29 +106,36 @@ __device__ __forceinline__ UnitGeom unit_geom(int a_src, int t, int row0, int64_
   return u;
 }
 
-__device__ __forceinline__ float unit_scale(const GemmParams& p, int64_t blk, float mean) {
-  const int64_t nb = (p.nw * p.kw + kB1 - 1) / kB1;
-  if (blk < 0 || blk >= nb) return 0.0f;
-  return dq_block_scale(__ldg(p.scale_codes + blk), __ldg(p.c2 + (blk >> 8)), mean);
-}
+// Raw per-unit scale data, fetched one iteration ahead of its use.
+struct UnitScale {
+  uint32_t e0, e1;   // scale codes of the unit's block and (generic path) of the next block
+  float c20, c21;    // their group constants
+  int32_t split;     // words before the block boundary (8 = one block), generic path only
+  int32_t valid;     // valid 8-code words (0 = unit outside the weight)
+};
 
-__device__ __forceinline__ void store_row_chunks(uint8_t* A, const UnitGeom& u, const uint32_t (&words)[8],
-                                                 const Nf4Lut& L0, const Nf4Lut& L1, int split_word,
-                                                 uint32_t valid_words) {
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    uint32_t o[4];
-    if ((uint32_t)j < valid_words) {
-      nf4_expand8(words[j], j < split_word ? L0 : L1, o);
-    } else {
-      o[0] = o[1] = o[2] = o[3] = 0u;
+template <bool GENERIC>
+__device__ __forceinline__ UnitScale fetch_scale(const GemmParams& p, const UnitGeom& u, int64_t nb) {
+  UnitScale r{0u, 0u, 0.0f, 0.0f, 8, 0};
+  if (u.n >= p.nw || u.kcol >= p.kw) return r;
+  const int64_t f0 = u.n * p.kw + u.kcol;
+  const int64_t blk = f0 >> 6;
+  r.e0 = __ldg(p.scale_codes + blk);
+  r.c20 = __ldg(p.c2 + (blk >> 8));
+  r.valid = 8;
+  if constexpr (GENERIC) {
+    r.split = (int32_t)((64 - (f0 & 63)) >> 3);
+    if (r.split < 8 && blk + 1 < nb) {
+      r.e1 = __ldg(p.scale_codes + blk + 1);
+      r.c21 = __ldg(p.c2 + ((blk + 1) >> 8));
     }
-    const uint32_t off = u.dst + (((uint32_t)j ^ u.swz) << 4);
-    *reinterpret_cast<uint4*>(A + off) = make_uint4(o[0], o[1], o[2], o[3]);
+    const int64_t vw = (p.kw - u.kcol) >> 3;
+    r.valid = (int32_t)(vw < 8 ? vw : 8);
   }
+  return r;
 }
 
-template <int BN>
+template <int BN, bool GENERIC>
 __global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_constant__ GemmParams p) {
   using C = Cfg<BN>;
   constexpr int S = C::kStages;
@@ -190,14 +198,14 @@ __global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_co
       if (lane == 0) {
         uint32_t bytes = C::kBBytes;
         const bool nf4 = (sg.a_src == kANf4K || sg.a_src == kANf4MN);
-        if (nf4 && !p.nf4_generic) bytes += kCodesBytes;
+        if (nf4 && !GENERIC) bytes += kCodesBytes;
         if (!nf4) bytes += C::kABytes;
         mbar_arrive_expect_tx(&full[s], bytes);
         const int k = sg.a_k0 + ip.kb * kBK;
         if (sg.a_src == kANf4K) {
-          if (!p.nf4_generic) tma_load_2d(stage_c(s), &p.maps[sg.a_map], k / 2, row0, &full[s]);
+          if (!GENERIC) tma_load_2d(stage_c(s), &p.maps[sg.a_map], k / 2, row0, &full[s]);
         } else if (sg.a_src == kANf4MN) {
-          if (!p.nf4_generic) tma_load_2d(stage_c(s), &p.maps[sg.a_map], row0 / 2, k, &full[s]);
+          if (!GENERIC) tma_load_2d(stage_c(s), &p.maps[sg.a_map], row0 / 2, k, &full[s]);
         } else if (sg.a_src == kATmaK) {
           tma_load_2d(stage_a(s), &p.maps[sg.a_map], k, row0, &full[s]);
         } else {
@@ -249,55 +257,70 @@ __global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_co
     __syncwarp();
   } else {
     // ------------------------------------------------------------------ dequant producer
-    const int t = threadIdx.x - 64;   // 0..127
+    // Two groups of four warps take alternate k-blocks; within a group thread t owns one
+    // 64-weight unit per k-block.
+    const int grp = (warp - 2) >> 2;          // 0: warps 2-5, 1: warps 6-9
+    const int t = (threadIdx.x - 64) & 127;
     bool ok = true;
     if (p.has_nf4) {
       const float mean = __ldg(p.mean);
-      for (int it = 0; it < n_iters && ok; ++it) {
-        const int s = it % S;
-        const uint32_t ph = (uint32_t)(it / S) & 1u;
+      const int64_t nb = (p.nw * p.kw + kB1 - 1) / kB1;
+      auto geom = [&](int it, bool& nf4, UnitGeom& u) {
         const IterPos ip = iter_pos(p, it, kb_begin, kb_end, first_split);
         const GemmSeg& sg = p.seg[ip.seg];
-        const bool nf4 = (sg.a_src == kANf4K || sg.a_src == kANf4MN);
-        UnitGeom u{};
+        nf4 = (sg.a_src == kANf4K || sg.a_src == kANf4MN);
+        if (nf4) u = unit_geom(sg.a_src, t, row0, (int64_t)sg.a_k0 + (int64_t)ip.kb * kBK);
+      };
+      bool nf4_next = false;
+      UnitGeom u_next{};
+      UnitScale sc_next{};
+      if (grp < n_iters) {
+        geom(grp, nf4_next, u_next);
+        if (nf4_next) sc_next = fetch_scale<GENERIC>(p, u_next, nb);
+      }
+      for (int it = grp; it < n_iters; it += 2) {
+        const int s = it % S;
+        const uint32_t ph = (uint32_t)(it / S) & 1u;
+        const bool nf4 = nf4_next;
+        const UnitGeom u = u_next;
+        const UnitScale sc = sc_next;
+        if (it + 2 < n_iters) {               // prefetch the next iteration's scales
+          geom(it + 2, nf4_next, u_next);
+          if (nf4_next) sc_next = fetch_scale<GENERIC>(p, u_next, nb);
+        }
         Nf4Lut L0, L1;
-        int split_word = 8;
-        uint32_t valid_words = 8;
         uint32_t words[8];
         if (nf4) {
-          const int64_t k = (int64_t)sg.a_k0 + (int64_t)ip.kb * kBK;
-          u = unit_geom(sg.a_src, t, row0, k);
-          const bool in_range = (u.n < p.nw) && (u.kcol < p.kw);
-          const int64_t f0 = u.n * p.kw + u.kcol;            // flat index of the unit's first weight
-          const int64_t blk0 = f0 >> 6;
-          float s0 = 0.0f, s1 = 0.0f;
-          if (in_range) {
-            s0 = unit_scale(p, blk0, mean);
-            if (p.nf4_generic) {
-              split_word = (int)((64 - (f0 & 63)) >> 3);     // words before the block boundary
-              if (split_word < 8) s1 = unit_scale(p, blk0 + 1, mean);
-              int64_t vw = (p.kw - u.kcol) >> 3;
-              valid_words = (uint32_t)(vw < 8 ? vw : 8);
-              const uint32_t* src = reinterpret_cast<const uint32_t*>(p.codes + (f0 >> 1));
+          nf4_lut_build(sc.valid ? dq_block_scale(sc.e0, sc.c20, mean) : 0.0f, L0);
+          if constexpr (GENERIC) {
+            if (sc.split < 8) nf4_lut_build(dq_block_scale(sc.e1, sc.c21, mean), L1);
+            const uint32_t* src = reinterpret_cast<const uint32_t*>(p.codes + ((u.n * p.kw + u.kcol) >> 1));
 #pragma unroll
-              for (int j = 0; j < 8; ++j) words[j] = ((uint32_t)j < valid_words) ? __ldg(src + j) : 0u;
-            }
-          } else {
-            valid_words = 0;
+            for (int j = 0; j < 8; ++j) words[j] = (j < sc.valid) ? __ldg(src + j) : 0u;
           }
-          nf4_lut_build(s0, L0);
-          if (split_word < 8) nf4_lut_build(s1, L1);
-          else L1 = L0;
         }
         if (!mbar_wait(&full[s], ph, abort_word, kErrWaitTma)) { ok = false; break; }
         if (nf4) {
-          if (!p.nf4_generic) {
+          uint8_t* A = stage_a(s);
+          if constexpr (!GENERIC) {
             const uint4* src = reinterpret_cast<const uint4*>(stage_c(s) + t * 32);
             const uint4 c0 = src[0], c1 = src[1];
             words[0] = c0.x; words[1] = c0.y; words[2] = c0.z; words[3] = c0.w;
             words[4] = c1.x; words[5] = c1.y; words[6] = c1.z; words[7] = c1.w;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              uint32_t o[4];
+              nf4_expand8(words[j], L0, o);
+              *reinterpret_cast<uint4*>(A + u.dst + (((uint32_t)j ^ u.swz) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              uint32_t o[4] = {0u, 0u, 0u, 0u};
+              if (j < sc.valid) nf4_expand8(words[j], j < sc.split ? L0 : L1, o);
+              *reinterpret_cast<uint4*>(A + u.dst + (((uint32_t)j ^ u.swz) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+            }
           }
-          store_row_chunks(stage_a(s), u, words, L0, L1, split_word, valid_words);
           fence_proxy_async_smem();
         }
         __syncwarp();
@@ -305,14 +328,17 @@ __global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_co
       }
     }
     // ------------------------------------------------------------------ epilogue
-    if (mbar_wait(accfull, 0u, abort_word, kErrWaitMma)) {
+    // Each group reads its half of the accumulator columns (group 0 all of them when BN < 64).
+    constexpr int kChunk = BN < 32 ? BN : 32;
+    const int c_begin = (BN < 64) ? 0 : grp * (BN / 2);
+    const int c_end = (BN < 64) ? (grp == 0 ? BN : 0) : c_begin + BN / 2;
+    if (c_begin < c_end && mbar_wait(accfull, 0u, abort_word, kErrWaitMma)) {
       tc_fence_after();
       const int q = warp & 3;
       const int row = row0 + 32 * q + lane;
       const bool row_ok = row < p.rows;
-      constexpr int kChunk = BN < 32 ? BN : 32;
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += kChunk) {
+      for (int c0 = c_begin; c0 < c_end; c0 += kChunk) {
         uint32_t r[32];
         const uint32_t taddr = tmem_acc + ((uint32_t)(32 * q) << 16) + (uint32_t)c0;
         if constexpr (kChunk == 32) tmem_ld_32x32b_x32(taddr, r);
@@ -326,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_co
             const int col = col0 + c0 + j;
             if (col < p.cols) out[(int64_t)col * p.ld_out + row] = f32_to_bf16_bits(__uint_as_float(r[j]));
           }
-        } else if (p.epi == kEpiF32T) {
+        } else {
           float* out = reinterpret_cast<float*>(p.out) + (int64_t)split * p.split_stride;
 #pragma unroll
           for (int j = 0; j < kChunk; ++j) {
@@ -346,30 +372,35 @@ __global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_co
   }
 }
 
-template <int BN>
+template <int BN, bool GENERIC>
 static cudaError_t launch_bn(const GemmParams& p, cudaStream_t st) {
   using C = Cfg<BN>;
   static bool configured = false;   // per process; the attribute is per function, not per device
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(qlora_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(qlora_gemm_kernel<BN, GENERIC>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     configured = true;
   }
   dim3 grid((p.rows + kBM - 1) / kBM, (p.cols + BN - 1) / BN, p.splits);
-  qlora_gemm_kernel<BN><<<grid, kThreads, C::kSmemBytes, st>>>(p);
+  qlora_gemm_kernel<BN, GENERIC><<<grid, kThreads, C::kSmemBytes, st>>>(p);
   return cudaGetLastError();
 }
 
-cudaError_t launch_gemm(const GemmParams& p, int bn, cudaStream_t st) {
+template <bool GENERIC>
+static cudaError_t launch_gemm_g(const GemmParams& p, int bn, cudaStream_t st) {
   switch (bn) {
-    case 16: return launch_bn<16>(p, st);
-    case 32: return launch_bn<32>(p, st);
-    case 64: return launch_bn<64>(p, st);
-    case 128: return launch_bn<128>(p, st);
-    case 256: return launch_bn<256>(p, st);
+    case 16: return launch_bn<16, GENERIC>(p, st);
+    case 32: return launch_bn<32, GENERIC>(p, st);
+    case 64: return launch_bn<64, GENERIC>(p, st);
+    case 128: return launch_bn<128, GENERIC>(p, st);
+    case 256: return launch_bn<256, GENERIC>(p, st);
     default: return cudaErrorInvalidValue;
   }
+}
+
+cudaError_t launch_gemm(const GemmParams& p, int bn, cudaStream_t st) {
+  return p.nf4_generic ? launch_gemm_g<true>(p, bn, st) : launch_gemm_g<false>(p, bn, st);
 }
 
 // ---------------------------------------------------------------------------------------
