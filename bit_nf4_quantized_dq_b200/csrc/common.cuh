@@ -77,23 +77,45 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
       : "memory");
   return ok != 0;
 }
-// Bounded wait: returns false (and raises `flag` in the device error word and in the
-// CTA-local abort word) if the phase did not complete within kWaitLimitNs of wall-clock
-// time, or if another role of the CTA has already aborted.
+// try_wait with acquire semantics at cluster scope (for phases completed by another CTA).
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait, called by all 32 lanes of a warp: returns false (and raises `flag` in the
+// device error word and in the CTA-local abort word) if the phase did not complete within
+// kWaitLimitNs of wall-clock time, or if another role of the CTA has already aborted.  The
+// result is the same for every lane, so loops that stop on failure stay warp-uniform.
+template <bool CLUSTER_ACQUIRE = false>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile uint32_t* abort_word,
                                           uint32_t flag) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait_sleep(bar, parity, 1000u)) return true;
-    if ((i & 15u) == 0u) {
-      if (*abort_word) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) break;
+  auto poll = [&]() { return CLUSTER_ACQUIRE ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
+  bool ok = poll();
+  if (!ok) {
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t i = 1;; ++i) {
+      if (CLUSTER_ACQUIRE ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait_sleep(bar, parity, 1000u)) {
+        ok = true;
+        break;
+      }
+      if ((i & 15u) == 0u) {
+        if (*abort_word) break;
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+          *abort_word = 1u;
+          atomicOr(&g_error_word, flag);
+          break;
+        }
+      }
     }
   }
-  *abort_word = 1u;
-  atomicOr(&g_error_word, flag);
-  return false;
+  return __all_sync(0xFFFFFFFFu, ok);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -109,6 +131,14 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
       "[%4];" ::"r"(smem_u32(smem_dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
       : "memory");
+}
+
+// Bring a tensor tile into L2 ahead of its load (no shared memory, no completion signal).
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* map, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y)
+               : "memory");
 }
 
 // generic-proxy shared-memory writes -> visible to the async proxy (UMMA operand reads)

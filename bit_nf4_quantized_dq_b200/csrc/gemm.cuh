@@ -36,11 +36,14 @@ struct Cfg {
   static constexpr int kBBytes = BN * kBK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes + kCodesBytes;
   static constexpr int kStagesRaw = (220 * 1024 - 2048) / kStageBytes;
-  static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
+  // Even: the two producer groups take alternate k-blocks, so each group must own whole
+  // stages and wait on every phase of their barriers (a parity wait that skips a phase can
+  // pass early).
+  static constexpr int kStages = (kStagesRaw > 8 ? 8 : kStagesRaw) & ~1;
   static constexpr int kTmemCols = BN <= 32 ? 32 : BN;
   static constexpr int kBarrierBytes = 256;
   static constexpr int kSmemBytes = kStages * kStageBytes + kBarrierBytes + 1024;
-  static_assert(kStages >= 2, "pipeline too shallow");
+  static_assert(kStages >= 2 && kStages % 2 == 0, "pipeline too shallow, or odd");
   static_assert(kBBytes % 1024 == 0, "B tile must keep 1024-byte alignment");
 };
 
@@ -214,6 +217,16 @@ __global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_co
         }
         tma_load_2d(stage_b(s), &p.maps[sg.b_map], sg.b_k0 + ip.kb * kBK, col0, &full[s]);
         last_issue[s] = it;
+        // L2 prefetch one ring ahead: many CTAs stream the same B tiles at about the same
+        // time, so the loads of the next ring pass then hit in L2 instead of waiting on DRAM.
+        if (it + S < n_iters) {
+          const IterPos pp = iter_pos(p, it + S, kb_begin, kb_end, first_split);
+          const GemmSeg& pg = p.seg[pp.seg];
+          const int pk = pg.a_k0 + pp.kb * kBK;
+          tma_prefetch_l2_2d(&p.maps[pg.b_map], pg.b_k0 + pp.kb * kBK, col0);
+          if (pg.a_src == kANf4K && !GENERIC) tma_prefetch_l2_2d(&p.maps[pg.a_map], pk / 2, row0);
+          else if (pg.a_src == kANf4MN && !GENERIC) tma_prefetch_l2_2d(&p.maps[pg.a_map], row0 / 2, pk);
+        }
       }
       __syncwarp();
     }
@@ -389,6 +402,7 @@ static cudaError_t launch_bn(const GemmParams& p, cudaStream_t st) {
 
 template <bool GENERIC>
 static cudaError_t launch_gemm_g(const GemmParams& p, int bn, cudaStream_t st) {
+  if (p.b_box_rows != bn) return cudaErrorInvalidValue;   // each B box must fill exactly one B tile
   switch (bn) {
     case 16: return launch_bn<16, GENERIC>(p, st);
     case 32: return launch_bn<32, GENERIC>(p, st);

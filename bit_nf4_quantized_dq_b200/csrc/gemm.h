@@ -41,6 +41,7 @@ struct GemmParams {
   int32_t rows, cols;            // valid extent of D: rows on the UMMA M side, cols on the N side
   int32_t splits, kb_per_split;  // segment 0 is split over blockIdx.z; later segments run in split 0
   int32_t has_nf4, nf4_generic;  // NF4 producer present; codes fetched without TMA (K % 64 != 0)
+  int32_t b_box_rows;            // rows of every B-operand TMA box (checked against the kernel's tile)
   // NF4 operand: codes / scale codes / group constants / mean of W [nw][kw]
   const uint8_t* codes;
   const uint8_t* scale_codes;

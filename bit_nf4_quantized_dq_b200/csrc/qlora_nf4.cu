@@ -9,6 +9,7 @@
 #include "qlora_nf4.h"
 #include "codec.cuh"
 #include "gemm.cuh"
+#include "gemm2sm.cuh"
 #include "lowrank.cuh"
 
 namespace {
@@ -259,6 +260,16 @@ int run_lowrank(const void* a_base, bool a_mn, int64_t a_inner, int64_t a_outer,
   return QNF4_OK;
 }
 
+// The fused GEMMs run on one CTA per tile; kPairTiles switches 256-token tiles to CTA pairs
+// (cta_group::2, gemm2sm.cuh).  Rows of each B-operand TMA box: a CTA of a pair loads half of
+// the 256-token tile.
+constexpr bool kPairTiles = false;
+int b_box_rows(int bn) { return (kPairTiles && bn == 256) ? 128 : bn; }
+
+cudaError_t launch_fused(const qnf4::GemmParams& gp, int bn, cudaStream_t st) {
+  return (kPairTiles && bn == 256) ? qnf4::launch_gemm2(gp, st) : qnf4::launch_gemm(gp, bn, st);
+}
+
 int nf4_operand(qnf4::GemmParams& gp, const uint8_t* codes, const uint8_t* scale_codes, const float* c2,
                 const float* mean, int64_t N, int64_t K) {
   gp.has_nf4 = 1;
@@ -390,10 +401,12 @@ int qlora_linear_fwd(const uint16_t* x, int64_t M, int64_t K, int64_t N, const u
     if (!generic) {
       if (int rc = make_map(&gp.maps[0], codes, false, K / 2, N, K / 2, 32, 128)) return rc;
     }
-    if (int rc = make_map(&gp.maps[1], x, true, K, M, K * 2, 64, plan.bn)) return rc;
+    const int bbox = b_box_rows(plan.bn);
+    if (int rc = make_map(&gp.maps[1], x, true, K, M, K * 2, 64, bbox)) return rc;
     if (int rc = make_map(&gp.maps[2], B, true, r, N, (uint64_t)r * 2, 64, 128)) return rc;
-    if (int rc = make_map(&gp.maps[3], w.thi, true, r, M, (uint64_t)r * 2, 64, plan.bn)) return rc;
-    if (int rc = make_map(&gp.maps[4], w.tlo, true, r, M, (uint64_t)r * 2, 64, plan.bn)) return rc;
+    if (int rc = make_map(&gp.maps[3], w.thi, true, r, M, (uint64_t)r * 2, 64, bbox)) return rc;
+    if (int rc = make_map(&gp.maps[4], w.tlo, true, r, M, (uint64_t)r * 2, 64, bbox)) return rc;
+    gp.b_box_rows = bbox;
     nf4_operand(gp, codes, scale_codes, c2, mean, N, K);
     gp.nseg = 3;
     gp.seg[0] = qnf4::GemmSeg{kblocks(K), k16_last(K), qnf4::kANf4K, 0, 1, 0, 0, 0};
@@ -413,7 +426,7 @@ int qlora_linear_fwd(const uint16_t* x, int64_t M, int64_t K, int64_t N, const u
       gp.out = y;
       gp.ld_out = N;
     }
-    cudaError_t e = qnf4::launch_gemm(gp, plan.bn, st);
+    cudaError_t e = launch_fused(gp, plan.bn, st);
     if (e != cudaSuccess) return cuda_fail(e, "fused forward launch");
     if (plan.splits > 1) {
       e = qnf4::launch_reduce_splits_bf16(w.part, plan.splits, M * N, M, N, N, y, N, st);
@@ -496,10 +509,12 @@ int qlora_linear_bwd(const uint16_t* dY, const uint16_t* x, const float* t_saved
     if (!generic) {
       if (int rc = make_map(&gp.maps[0], codes, false, K / 2, N, K / 2, 64, 64)) return rc;
     }
-    if (int rc = make_map(&gp.maps[1], dY, true, N, M, N * 2, 64, plan.bn)) return rc;
+    const int bbox = b_box_rows(plan.bn);
+    if (int rc = make_map(&gp.maps[1], dY, true, N, M, N * 2, 64, bbox)) return rc;
     if (int rc = make_map(&gp.maps[2], A, true, K, r, K * 2, 64, 64)) return rc;
-    if (int rc = make_map(&gp.maps[3], w.uhi, true, r, M, (uint64_t)r * 2, 64, plan.bn)) return rc;
-    if (int rc = make_map(&gp.maps[4], w.ulo, true, r, M, (uint64_t)r * 2, 64, plan.bn)) return rc;
+    if (int rc = make_map(&gp.maps[3], w.uhi, true, r, M, (uint64_t)r * 2, 64, bbox)) return rc;
+    if (int rc = make_map(&gp.maps[4], w.ulo, true, r, M, (uint64_t)r * 2, 64, bbox)) return rc;
+    gp.b_box_rows = bbox;
     nf4_operand(gp, codes, scale_codes, c2, mean, N, K);
     gp.nseg = 3;
     gp.seg[0] = qnf4::GemmSeg{kblocks(N), k16_last(N), qnf4::kANf4MN, 0, 1, 0, 0, 0};
@@ -519,7 +534,7 @@ int qlora_linear_bwd(const uint16_t* dY, const uint16_t* x, const float* t_saved
       gp.out = dX;
       gp.ld_out = K;
     }
-    e = qnf4::launch_gemm(gp, plan.bn, st);
+    e = launch_fused(gp, plan.bn, st);
     if (e != cudaSuccess) return cuda_fail(e, "fused dX launch");
     if (plan.splits > 1) {
       e = qnf4::launch_reduce_splits_bf16(w.partX, plan.splits, M * K, M, K, K, dX, K, st);

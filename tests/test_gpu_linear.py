@@ -125,3 +125,13 @@ def test_zero_adapter_b_gives_base_gemm():
     ow = oracle_weight(W)
     ref = oracle_linear(inp["x"], ow["w_deq"], inp["A"], B0, inp["dY"], 0.25)
     assert_within_tolerance(got["y"], ref["y"], "B=0 y")
+
+
+@pytest.mark.parametrize("M", [24, 48, 100, 200, 300, 520])
+def test_token_counts_cover_every_tile_width(M):
+    """Token counts that select each token-tile width of the fused GEMMs (16 ... 256, one-CTA
+    and CTA-pair kernels), on an aligned and on a K % 64 != 0 weight."""
+    for (N, K, seed) in ((640, 1024, 51), (520, 1000, 52)):
+        W = synth.normal_bf16((N, K), 0.02, seed)
+        inp = synth.linear_inputs(M, N, K, 32, seed + 100)
+        _check(W, inp["x"], inp["A"], inp["B"], inp["dY"], 0.5, tag=f"M={M} N={N} K={K}")
