@@ -31,6 +31,7 @@ SIGNATURES = {
     "nf4_quantize_workspace_bytes": (c_size_t, [c_int64]),
     "nf4_quantize_dq": (c_int, [c_void_p, c_int64, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                 c_size_t, c_void_p]),
+    "nf4_quantize_dq_noalloc": (c_int, [c_void_p, c_int64, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
     "nf4_dequant": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_void_p, c_void_p]),
     "qlora_linear_fwd_workspace_bytes": (c_size_t, [c_int64, c_int64, c_int64, c_int]),
     "qlora_linear_fwd": (c_int, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_void_p, c_void_p,
@@ -154,6 +155,28 @@ def nf4_quantize_dq(W: torch.Tensor, workspace: Optional[torch.Tensor] = None) -
     _check(L.nf4_quantize_dq(_ptr(W), numel, _ptr(codes), _ptr(scale_codes), _ptr(c2), _ptr(mean),
                              _ptr(workspace), workspace.numel(), _stream()), "nf4_quantize_dq")
     return NF4Tensor(codes, scale_codes, c2, mean, W.shape)
+
+
+def nf4_quantize_dq_noalloc(W: torch.Tensor, out: Optional[NF4Tensor] = None) -> NF4Tensor:
+    """nf4_quantize_dq without a workspace: the library's static scratch holds the absmax and
+    group sums (numel <= NOALLOC_MAX_NUMEL; overlapping calls on one device race on it).  Pass
+    `out` to write into existing buffers, so that the call itself allocates nothing."""
+    W = _bf16_bits(W)
+    _require_cuda(W)
+    numel = W.numel()
+    if out is None:
+        nb = (numel + 63) // 64
+        dev = W.device
+        out = NF4Tensor(torch.empty(32 * nb, dtype=torch.uint8, device=dev),
+                        torch.empty(nb, dtype=torch.uint8, device=dev),
+                        torch.empty((nb + 255) // 256, dtype=torch.float32, device=dev),
+                        torch.empty(1, dtype=torch.float32, device=dev), W.shape)
+    _check(lib().nf4_quantize_dq_noalloc(_ptr(W), numel, _ptr(out.codes), _ptr(out.scale_codes), _ptr(out.c2),
+                                         _ptr(out.mean), _stream()), "nf4_quantize_dq_noalloc")
+    return out
+
+
+NOALLOC_MAX_NUMEL = 1 << 28   # QNF4_NOALLOC_MAX_NUMEL
 
 
 def nf4_dequant(q: NF4Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:

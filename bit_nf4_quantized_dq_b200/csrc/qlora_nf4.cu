@@ -4,6 +4,7 @@
 #include <cstdio>
 #include <algorithm>
 #include <cstring>
+#include <mutex>
 #include <string>
 
 #include "qlora_nf4.h"
@@ -285,6 +286,49 @@ int nf4_operand(qnf4::GemmParams& gp, const uint8_t* codes, const uint8_t* scale
 
 }  // namespace
 
+// ---------------------------------------------------------------------------------------
+// Library-owned quantization scratch (nf4_quantize_dq_noalloc)
+// ---------------------------------------------------------------------------------------
+// For callers that cannot allocate device memory when they quantize (a host program handed
+// only the weight and output buffers, or a runtime whose device memory is all reserved for
+// its own pool), the absmax and group-sum scratch of the quantizer lives in this static
+// array: QNF4_NOALLOC_MAX_NUMEL / 64 fp32 absmax values, then the float64 group sums.  The
+// CUDA runtime reserves it on each device when it loads this module there.
+namespace {
+constexpr int64_t kNoAllocBlocks = QNF4_NOALLOC_MAX_NUMEL / 64;
+constexpr int64_t kNoAllocGroups = (kNoAllocBlocks + 255) / 256;
+constexpr size_t kNoAllocAbsmaxBytes = (size_t)kNoAllocBlocks * 4;
+constexpr size_t kNoAllocScratchBytes = kNoAllocAbsmaxBytes + (size_t)kNoAllocGroups * 8;
+static_assert(QNF4_NOALLOC_MAX_NUMEL % 64 == 0 && kNoAllocAbsmaxBytes % 256 == 0, "scratch layout");
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_quant_scratch[kNoAllocScratchBytes];
+
+namespace {
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_scratch[kNoAllocMaxDevices];   // device address of g_quant_scratch, per device
+
+// One-time set-up per device: with that device current, look up the scratch's address.
+int noalloc_scratch(void** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kNoAllocMaxDevices)
+    return fail(QNF4_ERR_UNSUPPORTED, "device ordinal %d: the static scratch supports devices 0..%d", dev,
+                kNoAllocMaxDevices - 1);
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_scratch[dev]) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_quant_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the quantization scratch");
+    g_noalloc_scratch[dev] = ptr;
+  }
+  *out = g_noalloc_scratch[dev];
+  return QNF4_OK;
+}
+}  // namespace
+
 extern "C" {
 
 int qnf4_version(void) { return 100; }
@@ -326,6 +370,30 @@ int nf4_quantize_dq(const uint16_t* W, int64_t numel, uint8_t* codes, uint8_t* s
   const int64_t nb = (numel + 63) / 64;
   float* absmax = static_cast<float*>(workspace);
   double* gsum = reinterpret_cast<double*>(static_cast<char*>(workspace) + align_up((size_t)nb * 4, 256));
+  cudaError_t e = qnf4::launch_quantize(W, numel, codes, scale_codes, c2, mean, absmax, gsum,
+                                        static_cast<cudaStream_t>(stream), 0);
+  if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
+  return QNF4_OK;
+}
+
+int nf4_quantize_dq_noalloc(const uint16_t* W, int64_t numel, uint8_t* codes, uint8_t* scale_codes, float* c2,
+                            float* mean, void* stream) {
+  g_last_error.clear();
+  if (!W || !codes || !scale_codes || !c2 || !mean) return fail(QNF4_ERR_INVALID, "NULL pointer");
+  if (numel <= 0) return fail(QNF4_ERR_INVALID, "numel must be positive");
+  if (numel > QNF4_NOALLOC_MAX_NUMEL)
+    return fail(QNF4_ERR_UNSUPPORTED,
+                "numel %lld is above the static scratch limit of %lld weights; use nf4_quantize_dq with a workspace",
+                (long long)numel, (long long)QNF4_NOALLOC_MAX_NUMEL);
+  if (!aligned(W, 16) || !aligned(codes, 16) || !aligned(scale_codes, 8))
+    return fail(QNF4_ERR_UNSUPPORTED, "alignment: W and codes 16 B, scale_codes 8 B");
+  if (int rc = check_arch()) return rc;
+  void* scratch = nullptr;
+  if (int rc = noalloc_scratch(&scratch)) return rc;
+  // Same carving as nf4_quantize_dq's workspace; both parts are written before they are read.
+  const int64_t nb = (numel + 63) / 64;
+  float* absmax = static_cast<float*>(scratch);
+  double* gsum = reinterpret_cast<double*>(static_cast<char*>(scratch) + align_up((size_t)nb * 4, 256));
   cudaError_t e = qnf4::launch_quantize(W, numel, codes, scale_codes, c2, mean, absmax, gsum,
                                         static_cast<cudaStream_t>(stream), 0);
   if (e != cudaSuccess) return cuda_fail(e, "quantize launch");

@@ -12,7 +12,8 @@
  * Conventions for every entry point:
  *  - Every pointer is a DEVICE pointer owned by the caller, except where stated.  The library
  *    never allocates device memory and keeps no state between calls other than the device
- *    error word (see qnf4_device_error).
+ *    error word (see qnf4_device_error) and the static scratch array of
+ *    nf4_quantize_dq_noalloc.
  *  - bf16 tensors are passed as uint16_t bit patterns, row-major, densely packed.
  *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every call is
  *    stream-ordered and asynchronous: it returns after enqueueing its kernels.  Device-side
@@ -85,6 +86,39 @@ int qnf4_device_error(void* stream, uint32_t* word);
 size_t nf4_quantize_workspace_bytes(int64_t numel);
 int nf4_quantize_dq(const uint16_t* W, int64_t numel, uint8_t* codes, uint8_t* scale_codes, float* c2,
                     float* mean, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * NF4 blockwise quantization with double quantization, without a workspace argument.
+ * The method has no counterpart to this entry point: it is a calling convention of this
+ * library, and computes exactly what nf4_quantize_dq computes (bit-identical outputs).
+ *
+ * Meant for callers that cannot allocate device memory at the point of the call: a host
+ * program or plug-in that is handed only the weight and the output buffers and has no device
+ * allocator of its own, or a runtime that reserved device memory for its own pool up front
+ * and has no way to lend a temporary buffer.  Such a caller cannot supply the workspace that
+ * nf4_quantize_dq needs, so the library keeps that scratch itself: one static device array,
+ * sized for numel <= QNF4_NOALLOC_MAX_NUMEL (2^28 weights: 16 MiB of per-block absmax plus
+ * 128 KiB of per-group float64 sums), which the CUDA runtime reserves on each device when it
+ * loads the library's kernels there.
+ *
+ *   W, codes, scale_codes, c2, mean : as for nf4_quantize_dq (same layouts and alignment).
+ *
+ *  - numel above QNF4_NOALLOC_MAX_NUMEL returns QNF4_ERR_UNSUPPORTED before any device work;
+ *    quantize larger weights with nf4_quantize_dq and a workspace.
+ *  - The first call on each device does a one-time set-up: with that device current it looks
+ *    up the device address of the scratch array.  Make that first call before any stream
+ *    capture begins.
+ *  - Nothing has to start at zero: every scratch element a call reads, the same call writes
+ *    first.
+ *  - There is one scratch array per device, shared by every call on that device.  Calls that
+ *    overlap in time (on different streams, or from different host threads without ordering)
+ *    race on it and produce wrong results: order them on one stream or synchronise between
+ *    them.
+ *  - Allocates nothing: no cudaMalloc, cudaFree or allocating library routine is called.
+ * ------------------------------------------------------------------------------------- */
+#define QNF4_NOALLOC_MAX_NUMEL 268435456LL
+int nf4_quantize_dq_noalloc(const uint16_t* W, int64_t numel, uint8_t* codes, uint8_t* scale_codes,
+                            float* c2, float* mean, void* stream);
 
 /* ---------------------------------------------------------------------------------------
  * NF4 + DQ -> bf16 dequantization (the standalone HBM stream).
