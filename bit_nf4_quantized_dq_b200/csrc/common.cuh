@@ -89,13 +89,12 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
       : "memory");
   return ok != 0;
 }
-// Bounded wait, called by all 32 lanes of a warp: returns false (and raises `flag` in the
-// device error word and in the CTA-local abort word) if the phase did not complete within
-// kWaitLimitNs of wall-clock time, or if another role of the CTA has already aborted.  The
-// result is the same for every lane, so loops that stop on failure stay warp-uniform.
+// Bounded wait by one thread: returns false (and raises `flag` in the device error word and in
+// the CTA-local abort word) if the phase did not complete within kWaitLimitNs of wall-clock
+// time, or if another role of the CTA has already aborted.
 template <bool CLUSTER_ACQUIRE = false>
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile uint32_t* abort_word,
-                                          uint32_t flag) {
+__device__ __forceinline__ bool mbar_wait_thread(uint64_t* bar, uint32_t parity, volatile uint32_t* abort_word,
+                                                 uint32_t flag) {
   auto poll = [&]() { return CLUSTER_ACQUIRE ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
   bool ok = poll();
   if (!ok) {
@@ -115,7 +114,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
       }
     }
   }
-  return __all_sync(0xFFFFFFFFu, ok);
+  return ok;
+}
+// The same, called by all 32 lanes of a warp; the result is the same for every lane, so loops
+// that stop on failure stay warp-uniform.
+template <bool CLUSTER_ACQUIRE = false>
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile uint32_t* abort_word,
+                                          uint32_t flag) {
+  return __all_sync(0xFFFFFFFFu, mbar_wait_thread<CLUSTER_ACQUIRE>(bar, parity, abort_word, flag));
 }
 
 // ---------------------------------------------------------------------------------------

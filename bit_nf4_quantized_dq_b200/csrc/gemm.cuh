@@ -15,9 +15,9 @@
 // with the fp32 intermediates t and u split into bf16 hi + lo parts so that the adapter
 // terms keep close to fp32 accuracy through bf16 tensor-core inputs.
 //
-// Warp roles (320 threads): warp 0 issues TMA loads, warp 1 allocates TMEM and issues MMAs,
-// warps 2-9 run the dequant producer (two groups of four warps on alternate k-blocks) and
-// then the epilogue (each group drains half of the accumulator columns).
+// Warp roles: warp 0 (and warps 10.. when kTmaWarps > 1) issue TMA loads, warp 1 allocates TMEM
+// and issues MMAs, warps 2-9 run the dequant producer (two groups of four warps on alternate
+// k-blocks) and then the epilogue (each group drains half of the accumulator columns).
 #pragma once
 
 #include "nf4_device.cuh"
@@ -27,7 +27,11 @@ namespace qnf4 {
 
 constexpr int kBM = 128;
 constexpr int kBK = 64;
-constexpr int kThreads = 320;   // TMA warp, MMA warp, two groups of four producer / epilogue warps
+// A bulk-tensor load holds the thread that issues it for a few hundred cycles, whatever the box
+// size, while loads from different warps proceed side by side: kTmaWarps warps share the loads,
+// warp w (warp 0, then warps 10, 11, ...) taking the k-blocks it with it % kTmaWarps == w.
+constexpr int kTmaWarps = 2;
+constexpr int kThreads = 320 + 32 * (kTmaWarps - 1);   // + MMA warp, two groups of four producer / epilogue warps
 constexpr int kCodesBytes = 4096;   // packed codes of one 128 x 64 weight tile
 
 template <int BN>
@@ -44,6 +48,7 @@ struct Cfg {
   static constexpr int kBarrierBytes = 256;
   static constexpr int kSmemBytes = kStages * kStageBytes + kBarrierBytes + 1024;
   static_assert(kStages >= 2 && kStages % 2 == 0, "pipeline too shallow, or odd");
+  static_assert(kStages % kTmaWarps == 0, "each TMA warp must own whole stages");
   static_assert(kBBytes % 1024 == 0, "B tile must keep 1024-byte alignment");
 };
 
@@ -138,6 +143,36 @@ __device__ __forceinline__ UnitScale fetch_scale(const GemmParams& p, const Unit
   return r;
 }
 
+// One k-block (64 deep) of MMAs: four 16-deep tcgen05.mma into the accumulator.  The
+// descriptors of consecutive 16-deep slices differ only in their start address (bits 0-13,
+// 16-byte units): 32 bytes along a K-major row, 2048 bytes (16 K rows of 128 bytes) down an
+// MN-major chunk.  Start addresses stay below 2^18, so the field never carries.
+template <int BN, bool A_MN>
+__device__ __forceinline__ void umma_kblock(uint32_t tmem_acc, uint32_t a_addr, uint32_t b_addr, uint32_t acc) {
+  constexpr uint32_t idesc = umma_idesc_bf16(kBM, BN, A_MN ? 1u : 0u, 0u);
+  const uint64_t a0 = A_MN ? umma_sdesc_sw128(a_addr, 8192u, 1024u) : umma_sdesc_sw128(a_addr, 16u, 1024u);
+  const uint64_t b0 = umma_sdesc_sw128(b_addr, 16u, 1024u);
+#pragma unroll
+  for (int k16 = 0; k16 < 4; ++k16) {
+    const uint64_t ad = a0 + (uint64_t)((A_MN ? 2048u : 32u) * (uint32_t)k16 >> 4);
+    const uint64_t bd = b0 + (uint64_t)(32u * (uint32_t)k16 >> 4);
+    umma_bf16(tmem_acc, ad, bd, idesc, k16 == 0 ? acc : 1u);
+  }
+}
+
+// The last k-block of a stretch whose depth is not a multiple of 64: nk16 < 4 slices.
+template <int BN>
+__device__ __noinline__ void umma_kblock_ragged(uint32_t tmem_acc, uint32_t a_addr, uint32_t b_addr, uint32_t acc,
+                                                bool a_mn, int nk16) {
+  const uint32_t idesc = umma_idesc_bf16(kBM, BN, a_mn ? 1u : 0u, 0u);
+  for (int k16 = 0; k16 < nk16; ++k16) {
+    const uint64_t ad = a_mn ? umma_sdesc_sw128(a_addr + (uint32_t)k16 * 2048u, 8192u, 1024u)
+                             : umma_sdesc_sw128(a_addr + (uint32_t)k16 * 32u, 16u, 1024u);
+    const uint64_t bd = umma_sdesc_sw128(b_addr + (uint32_t)k16 * 32u, 16u, 1024u);
+    umma_bf16(tmem_acc, ad, bd, idesc, (acc || k16 > 0) ? 1u : 0u);
+  }
+}
+
 template <int BN, bool GENERIC>
 __global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_constant__ GemmParams p) {
   using C = Cfg<BN>;
@@ -187,12 +222,13 @@ __global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_co
   auto stage_b = [&](int s) { return smem + s * C::kStageBytes + C::kABytes; };
   auto stage_c = [&](int s) { return smem + s * C::kStageBytes + C::kABytes + C::kBBytes; };
 
-  if (warp == 0) {
-    // ------------------------------------------------------------------ TMA producer
+  if (warp == 0 || warp >= 10) {
+    // ------------------------------------------------------------------ TMA producers
+    const int tw = (warp == 0) ? 0 : warp - 9;
     int last_issue[8];
     for (int s = 0; s < 8; ++s) last_issue[s] = -1;
     bool ok = true;
-    for (int it = 0; it < n_iters && ok; ++it) {
+    for (int it = tw; it < n_iters && ok; it += kTmaWarps) {
       const int s = it % S;
       const uint32_t ph = (uint32_t)(it / S) & 1u;
       if (!mbar_wait(&empty[s], ph ^ 1u, abort_word, kErrWaitEmpty)) { ok = false; break; }
@@ -204,30 +240,32 @@ __global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_co
         if (nf4 && !GENERIC) bytes += kCodesBytes;
         if (!nf4) bytes += C::kABytes;
         mbar_arrive_expect_tx(&full[s], bytes);
-        const int k = sg.a_k0 + ip.kb * kBK;
-        if (sg.a_src == kANf4K) {
-          if (!GENERIC) tma_load_2d(stage_c(s), &p.maps[sg.a_map], k / 2, row0, &full[s]);
-        } else if (sg.a_src == kANf4MN) {
-          if (!GENERIC) tma_load_2d(stage_c(s), &p.maps[sg.a_map], row0 / 2, k, &full[s]);
-        } else if (sg.a_src == kATmaK) {
-          tma_load_2d(stage_a(s), &p.maps[sg.a_map], k, row0, &full[s]);
-        } else {
-          tma_load_2d(stage_a(s), &p.maps[sg.a_map], row0, k, &full[s]);
-          tma_load_2d(stage_a(s) + 8192, &p.maps[sg.a_map], row0 + 64, k, &full[s]);
-        }
-        tma_load_2d(stage_b(s), &p.maps[sg.b_map], sg.b_k0 + ip.kb * kBK, col0, &full[s]);
         last_issue[s] = it;
-        // L2 prefetch one ring ahead: many CTAs stream the same B tiles at about the same
-        // time, so the loads of the next ring pass then hit in L2 instead of waiting on DRAM.
-        if (it + S < n_iters) {
-          const IterPos pp = iter_pos(p, it + S, kb_begin, kb_end, first_split);
-          const GemmSeg& pg = p.seg[pp.seg];
-          const int pk = pg.a_k0 + pp.kb * kBK;
-          tma_prefetch_l2_2d(&p.maps[pg.b_map], pg.b_k0 + pp.kb * kBK, col0);
-          if (pg.a_src == kANf4K && !GENERIC) tma_prefetch_l2_2d(&p.maps[pg.a_map], pk / 2, row0);
-          else if (pg.a_src == kANf4MN && !GENERIC) tma_prefetch_l2_2d(&p.maps[pg.a_map], row0 / 2, pk);
-        }
       }
+      __syncwarp();
+      // A bulk-tensor load holds its issuing thread for a few hundred cycles whatever the box
+      // size, so one thread issuing the k-block's two or three loads one after the other
+      // would pace the whole pipeline.  Lanes 0..2 each take one load and issue them as a
+      // single instruction: lane 0 the B tile, lanes 1 and 2 the A side.
+      const int k = sg.a_k0 + ip.kb * kBK;
+      int map = -1, cx = 0, cy = 0;
+      uint8_t* dst = nullptr;
+      if (lane == 0) {
+        map = sg.b_map; dst = stage_b(s); cx = sg.b_k0 + ip.kb * kBK; cy = col0;
+      } else if (lane == 1) {
+        if (sg.a_src == kANf4K) {
+          if (!GENERIC) { map = sg.a_map; dst = stage_c(s); cx = k / 2; cy = row0; }
+        } else if (sg.a_src == kANf4MN) {
+          if (!GENERIC) { map = sg.a_map; dst = stage_c(s); cx = row0 / 2; cy = k; }
+        } else if (sg.a_src == kATmaK) {
+          map = sg.a_map; dst = stage_a(s); cx = k; cy = row0;
+        } else {
+          map = sg.a_map; dst = stage_a(s); cx = row0; cy = k;
+        }
+      } else if (lane == 2 && sg.a_src == kATmaMN) {
+        map = sg.a_map; dst = stage_a(s) + 8192; cx = row0 + 64; cy = k;
+      }
+      if (map >= 0) tma_load_2d(dst, &p.maps[map], cx, cy, &full[s]);
       __syncwarp();
     }
     if (!ok && lane == 0) {
@@ -241,32 +279,36 @@ __global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_co
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
-    bool ok = true;
-    for (int it = 0; it < n_iters && ok; ++it) {
-      const int s = it % S;
-      const uint32_t ph = (uint32_t)(it / S) & 1u;
-      if (!mbar_wait(&full[s], ph, abort_word, kErrWaitTma)) { ok = false; break; }
-      if (p.has_nf4 && !mbar_wait(&prod[s], ph, abort_word, kErrWaitProducer)) { ok = false; break; }
-      tc_fence_after();
-      const IterPos ip = iter_pos(p, it, kb_begin, kb_end, first_split);
-      const GemmSeg& sg = p.seg[ip.seg];
-      if (lane == 0) {
+    // Lane 0 alone runs this loop.  The tensor pipe queues only about one MMA ahead, so every
+    // cycle the issuer spends between k-blocks shows up as pipe idle time: no warp-collective
+    // instruction here, one barrier wait per k-block, and a fully unrolled MMA sequence.
+    // The producers arrive on prod[s] only after they saw full[s] complete, so with a
+    // producer present prod[s] alone orders the MMAs after both the TMA data and the
+    // dequantized tile.
+    if (lane == 0) {
+      uint64_t* const ready = p.has_nf4 ? prod : full;
+      const uint32_t ready_err = p.has_nf4 ? kErrWaitProducer : kErrWaitTma;
+      for (int it = 0; it < n_iters; ++it) {
+        const int s = it % S;
+        const uint32_t ph = (uint32_t)(it / S) & 1u;
+        if (!mbar_wait_thread(&ready[s], ph, abort_word, ready_err)) break;
+        tc_fence_after();
+        const IterPos ip = iter_pos(p, it, kb_begin, kb_end, first_split);
+        const GemmSeg& sg = p.seg[ip.seg];
         const bool a_mn = (sg.a_src == kANf4MN || sg.a_src == kATmaMN);
-        const uint32_t idesc = umma_idesc_bf16(kBM, BN, a_mn ? 1u : 0u, 0u);
         const uint32_t a_addr = smem_u32(stage_a(s));
         const uint32_t b_addr = smem_u32(stage_b(s));
-        const int nk16 = ip.last ? sg.k16_last : 4;
-        for (int k16 = 0; k16 < nk16; ++k16) {
-          const uint64_t ad = a_mn ? umma_sdesc_sw128(a_addr + (uint32_t)k16 * 2048u, 8192u, 1024u)
-                                   : umma_sdesc_sw128(a_addr + (uint32_t)k16 * 32u, 16u, 1024u);
-          const uint64_t bd = umma_sdesc_sw128(b_addr + (uint32_t)k16 * 32u, 16u, 1024u);
-          umma_bf16(tmem_acc, ad, bd, idesc, (it > 0 || k16 > 0) ? 1u : 0u);
+        const uint32_t acc = it > 0 ? 1u : 0u;
+        if (!ip.last || sg.k16_last == 4) {
+          if (a_mn) umma_kblock<BN, true>(tmem_acc, a_addr, b_addr, acc);
+          else umma_kblock<BN, false>(tmem_acc, a_addr, b_addr, acc);
+        } else {
+          umma_kblock_ragged<BN>(tmem_acc, a_addr, b_addr, acc, a_mn, sg.k16_last);
         }
         umma_commit(&empty[s]);
       }
-      __syncwarp();
+      umma_commit(accfull);   // also on abort: lets the epilogue wait out in-flight MMAs
     }
-    if (lane == 0) umma_commit(accfull);   // also on abort: lets the epilogue wait out in-flight MMAs
     __syncwarp();
   } else {
     // ------------------------------------------------------------------ dequant producer
