@@ -21,7 +21,7 @@
 
 namespace qnf4 {
 
-constexpr int kThreads2 = 320;
+constexpr int kThreads2 = 352;   // TMA warps 0 and 10, MMA warp 1, producer / epilogue warps 2-9
 
 struct Cfg2 {
   static constexpr int BN = 256;                    // UMMA N (tokens per pair)
@@ -103,6 +103,21 @@ __device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
       : "memory");
 }
 
+// One k-block (64 deep) of pair MMAs (M = 256 over the two CTAs, N = 256): the descriptors of
+// consecutive 16-deep slices differ only in their start address field.
+template <bool A_MN>
+__device__ __forceinline__ void umma_kblock_pair(uint32_t tmem_acc, uint32_t a_addr, uint32_t b_addr, uint32_t acc) {
+  constexpr uint32_t idesc = umma_idesc_bf16(256, Cfg2::BN, A_MN ? 1u : 0u, 0u);
+  const uint64_t a0 = A_MN ? umma_sdesc_sw128(a_addr, 8192u, 1024u) : umma_sdesc_sw128(a_addr, 16u, 1024u);
+  const uint64_t b0 = umma_sdesc_sw128(b_addr, 16u, 1024u);
+#pragma unroll
+  for (int k16 = 0; k16 < 4; ++k16) {
+    const uint64_t ad = a0 + (uint64_t)((A_MN ? 2048u : 32u) * (uint32_t)k16 >> 4);
+    const uint64_t bd = b0 + (uint64_t)(32u * (uint32_t)k16 >> 4);
+    umma_bf16_pair(tmem_acc, ad, bd, idesc, k16 == 0 ? acc : 1u);
+  }
+}
+
 template <bool GENERIC>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
     qlora_gemm2_kernel(const __grid_constant__ GemmParams p) {
@@ -165,12 +180,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
   auto tstage_c = [&](int s) { return smem + s * C::kTStageBytes + C::kBBytes; };
   auto aslot = [&](int a) { return smem + ST * C::kTStageBytes + a * C::kABytes; };
 
-  if (warp == 0) {
+  if (warp == 0 || warp >= 10) {
     // ------------------------------------------------------------------ TMA (both CTAs)
+    // Two warps (0 and 10) take alternate k-blocks: a bulk-tensor load holds its issuing
+    // thread for a few hundred cycles whatever its size, while loads of different warps, and
+    // of different lanes of one instruction, proceed side by side.  Each k-block's loads go
+    // out as one instruction: lane 0 this CTA's half of the B tile, lane 1 the codes (or the
+    // A tile), lane 2 the second half of an MN-major A tile.  All use the pair form, which
+    // completes on any mbarrier of the pair: the even CTA's full[s], or this CTA's cfull[s].
+    const int tw = (warp == 0) ? 0 : 1;
     int last_issue[ST];
     for (int s = 0; s < ST; ++s) last_issue[s] = -1;
     bool ok = true;
-    for (int it = 0; it < n_iters && ok; ++it) {
+    for (int it = tw; it < n_iters && ok; it += 2) {
       const int s = it % ST, a = it % SA;
       const uint32_t ph = (uint32_t)(it / ST) & 1u, pa = (uint32_t)(it / SA) & 1u;
       if (!mbar_wait(&empty[s], ph ^ 1u, abort_word, kErrWaitEmpty)) { ok = false; break; }
@@ -178,30 +200,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
       const GemmSeg& sg = p.seg[ip.seg];
       const bool nf4 = (sg.a_src == kANf4K || sg.a_src == kANf4MN);
       if (!nf4 && !mbar_wait(&aempty[a], pa ^ 1u, abort_word, kErrWaitEmpty)) { ok = false; break; }
+      const uint32_t fbar = full_leader0 + (uint32_t)s * 8u;
       if (lane == 0) {
-        const uint32_t fbar = full_leader0 + (uint32_t)s * 8u;
         if (rank == 0) mbar_arrive_expect_tx(&full[s], 2u * (C::kBBytes + (nf4 ? 0u : (uint32_t)C::kABytes)));
-        const int k = sg.a_k0 + ip.kb * kBK;
-        if (nf4 && !GENERIC) {
-          mbar_arrive_expect_tx(&cfull[s], kCodesBytes);
-          if (sg.a_src == kANf4K) tma_load_2d(tstage_c(s), &p.maps[sg.a_map], k / 2, row0, &cfull[s]);
-          else tma_load_2d(tstage_c(s), &p.maps[sg.a_map], row0 / 2, k, &cfull[s]);
-        } else {
-          mbar_arrive(&cfull[s]);         // keeps the producers in step with the stages
-        }
-        if (sg.a_src == kATmaK) {
-          tma_load_2d_pair(aslot(a), &p.maps[sg.a_map], k, row0, fbar);
-        } else if (sg.a_src == kATmaMN) {
-          tma_load_2d_pair(aslot(a), &p.maps[sg.a_map], row0, k, fbar);
-          tma_load_2d_pair(aslot(a) + 8192, &p.maps[sg.a_map], row0 + 64, k, fbar);
-        }
-        tma_load_2d_pair(tstage_b(s), &p.maps[sg.b_map], sg.b_k0 + ip.kb * kBK, col0 + 128 * (int)rank, fbar);
+        if (nf4 && !GENERIC) mbar_arrive_expect_tx(&cfull[s], kCodesBytes);
+        else mbar_arrive(&cfull[s]);      // keeps the producers in step with the stages
         last_issue[s] = it;
       }
       __syncwarp();
+      const int k = sg.a_k0 + ip.kb * kBK;
+      int map = -1, cx = 0, cy = 0;
+      uint8_t* dst = nullptr;
+      uint32_t bar = fbar;
+      if (lane == 0) {
+        map = sg.b_map; dst = tstage_b(s); cx = sg.b_k0 + ip.kb * kBK; cy = col0 + 128 * (int)rank;
+      } else if (lane == 1) {
+        if (nf4) {
+          if (!GENERIC) {
+            map = sg.a_map; dst = tstage_c(s); bar = smem_u32(&cfull[s]);
+            if (sg.a_src == kANf4K) { cx = k / 2; cy = row0; } else { cx = row0 / 2; cy = k; }
+          }
+        } else if (sg.a_src == kATmaK) {
+          map = sg.a_map; dst = aslot(a); cx = k; cy = row0;
+        } else {
+          map = sg.a_map; dst = aslot(a); cx = row0; cy = k;
+        }
+      } else if (lane == 2 && sg.a_src == kATmaMN) {
+        map = sg.a_map; dst = aslot(a) + 8192; cx = row0 + 64; cy = k;
+      }
+      if (map >= 0) tma_load_2d_pair(dst, &p.maps[map], cx, cy, bar);
+      __syncwarp();
     }
     if (!ok && lane == 0) {
-      // drain this CTA's copies still in flight (the pair's B copies complete on the even
+      // drain this warp's copies still in flight (the pair's B copies complete on the even
       // CTA's barriers, which that CTA drains)
       for (int s = 0; s < ST; ++s)
         if (last_issue[s] >= 0) {
@@ -214,36 +245,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer (even CTA)
-    if (rank == 0) {
-      bool ok = true;
-      for (int it = 0; it < n_iters && ok; ++it) {
+    // Lane 0 of the even CTA alone runs this loop: the tensor pipe queues only about one MMA
+    // ahead, so the issuer keeps warp-collective instructions out of it and issues each
+    // k-block as one unrolled sequence.
+    if (rank == 0 && lane == 0) {
+      for (int it = 0; it < n_iters; ++it) {
         const int s = it % ST, a = it % SA;
         const uint32_t ph = (uint32_t)(it / ST) & 1u, pa = (uint32_t)(it / SA) & 1u;
-        if (!mbar_wait(&full[s], ph, abort_word, kErrWaitTma)) { ok = false; break; }
-        if (!mbar_wait(&prod[a], pa, abort_word, kErrWaitProducer)) { ok = false; break; }
+        if (!mbar_wait_thread(&full[s], ph, abort_word, kErrWaitTma)) break;
+        if (!mbar_wait_thread(&prod[a], pa, abort_word, kErrWaitProducer)) break;
         tc_fence_after();
         const IterPos ip = iter_pos(p, it, kb_begin, kb_end, first_split);
         const GemmSeg& sg = p.seg[ip.seg];
-        if (lane == 0) {
-          const bool a_mn = (sg.a_src == kANf4MN || sg.a_src == kATmaMN);
+        const bool a_mn = (sg.a_src == kANf4MN || sg.a_src == kATmaMN);
+        const uint32_t a_addr = smem_u32(aslot(a));
+        const uint32_t b_addr = smem_u32(tstage_b(s));
+        const uint32_t acc = it > 0 ? 1u : 0u;
+        if (!ip.last || sg.k16_last == 4) {
+          if (a_mn) umma_kblock_pair<true>(tmem_acc, a_addr, b_addr, acc);
+          else umma_kblock_pair<false>(tmem_acc, a_addr, b_addr, acc);
+        } else {
           const uint32_t idesc = umma_idesc_bf16(256, C::BN, a_mn ? 1u : 0u, 0u);
-          const uint32_t a_addr = smem_u32(aslot(a));
-          const uint32_t b_addr = smem_u32(tstage_b(s));
-          const int nk16 = ip.last ? sg.k16_last : 4;
-          for (int k16 = 0; k16 < nk16; ++k16) {
+          for (int k16 = 0; k16 < sg.k16_last; ++k16) {
             const uint64_t ad = a_mn ? umma_sdesc_sw128(a_addr + (uint32_t)k16 * 2048u, 8192u, 1024u)
                                      : umma_sdesc_sw128(a_addr + (uint32_t)k16 * 32u, 16u, 1024u);
             const uint64_t bd = umma_sdesc_sw128(b_addr + (uint32_t)k16 * 32u, 16u, 1024u);
-            umma_bf16_pair(tmem_acc, ad, bd, idesc, (it > 0 || k16 > 0) ? 1u : 0u);
+            umma_bf16_pair(tmem_acc, ad, bd, idesc, (acc || k16 > 0) ? 1u : 0u);
           }
-          umma_commit_pair(&empty[s]);
-          umma_commit_pair(&aempty[a]);
         }
-        __syncwarp();
+        umma_commit_pair(&empty[s]);
+        umma_commit_pair(&aempty[a]);
       }
-      if (lane == 0) umma_commit_pair(accfull);   // also on abort: in-flight MMAs drain first
-      __syncwarp();
+      umma_commit_pair(accfull);   // also on abort: in-flight MMAs drain first
     }
+    __syncwarp();
   } else {
     // ------------------------------------------------------------------ dequant producer
     // Two groups of four warps take alternate k-blocks; within a group thread t owns one
