@@ -211,35 +211,58 @@ __global__ void __launch_bounds__(256) dq_groups_kernel(const float* __restrict_
 }
 
 // ---------------------------------------------------------------------------------------
-// D: standalone dequant, one thread per block of 64: two 16-byte code loads, the block's
-// bf16 table, eight 16-byte stores.
+// D: standalone dequant, one thread per block of 64 (two 16-byte code loads, the block's bf16
+// table).  A warp's 32 blocks are one contiguous 4 KB of output: the expanded rows go to
+// shared memory first (16-byte chunk j of block l at chunk position j ^ (l & 7), so that
+// neither the writes nor the reads conflict), then the warp stores 512 contiguous bytes per
+// instruction.  Warps whose blocks reach past the end use per-thread stores.
 // ---------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint8_t* __restrict__ codes,
                                                           const uint8_t* __restrict__ scale_codes,
                                                           const float* __restrict__ c2,
                                                           const float* __restrict__ mean_p, int64_t numel,
                                                           int64_t nb, uint16_t* __restrict__ out) {
-  const int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (b >= nb) return;
-  const float scale = dq_block_scale(__ldg(scale_codes + b), __ldg(c2 + (b >> 8)), __ldg(mean_p));
-  Nf4Lut L;
-  nf4_lut_build(scale, L);
-  const uint4* src = reinterpret_cast<const uint4*>(codes + b * 32);
-  const uint4 c0 = __ldg(src), c1 = __ldg(src + 1);
-  const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-  const int64_t e0 = b * kB1;
-  if (e0 + kB1 <= numel) {
-    uint4* dst = reinterpret_cast<uint4*>(out + e0);
+  __shared__ uint4 stage[8][32 * 8];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t b0 = (int64_t)blockIdx.x * blockDim.x + warp * 32;   // first block of this warp
+  const int64_t b = b0 + lane;
+  if (b0 >= nb) return;                                             // whole warps leave together
+  const bool whole = (b0 + 32) * kB1 <= numel;                      // implies b0 + 32 <= nb
+  uint32_t w[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  Nf4Lut L{};
+  if (b < nb) {
+    const float scale = dq_block_scale(__ldg(scale_codes + b), __ldg(c2 + (b >> 8)), __ldg(mean_p));
+    nf4_lut_build(scale, L);
+    const uint4* src = reinterpret_cast<const uint4*>(codes + b * 32);
+    const uint4 c0 = __ldg(src), c1 = __ldg(src + 1);
+    w[0] = c0.x; w[1] = c0.y; w[2] = c0.z; w[3] = c0.w;
+    w[4] = c1.x; w[5] = c1.y; w[6] = c1.z; w[7] = c1.w;
+  }
+  if (whole) {
+    uint4* row = stage[warp];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       uint32_t o[4];
       nf4_expand8(w[j], L, o);
-      dst[j] = make_uint4(o[0], o[1], o[2], o[3]);
+      row[lane * 8 + (j ^ (lane & 7))] = make_uint4(o[0], o[1], o[2], o[3]);
     }
-  } else {
-    for (int j = 0; j < 8; ++j) {
-      uint32_t o[4];
-      nf4_expand8(w[j], L, o);
+    __syncwarp();
+    uint4* dst = reinterpret_cast<uint4*>(out + b0 * kB1);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int q = i * 32 + lane, lb = q >> 3, j = q & 7;
+      dst[q] = row[lb * 8 + (j ^ (lb & 7))];
+    }
+    return;
+  }
+  if (b >= nb) return;
+  const int64_t e0 = b * kB1;
+  for (int j = 0; j < 8; ++j) {
+    uint32_t o[4];
+    nf4_expand8(w[j], L, o);
+    if (e0 + 8 * j + 8 <= numel) {
+      *reinterpret_cast<uint4*>(out + e0 + 8 * j) = make_uint4(o[0], o[1], o[2], o[3]);
+    } else {
       for (int i = 0; i < 8; ++i) {
         const int64_t e = e0 + 8 * j + i;
         if (e < numel) out[e] = (uint16_t)((o[i >> 1] >> (16 * (i & 1))) & 0xFFFFu);

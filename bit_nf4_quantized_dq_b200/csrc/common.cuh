@@ -92,7 +92,8 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
 // Bounded wait by one thread: returns false (and raises `flag` in the device error word and in
 // the CTA-local abort word) if the phase did not complete within kWaitLimitNs of wall-clock
 // time, or if another role of the CTA has already aborted.
-template <bool CLUSTER_ACQUIRE = false>
+// SPIN polls without a suspend hint (for hand-offs on the critical path of every k-block).
+template <bool CLUSTER_ACQUIRE = false, bool SPIN = false>
 __device__ __forceinline__ bool mbar_wait_thread(uint64_t* bar, uint32_t parity, volatile uint32_t* abort_word,
                                                  uint32_t flag) {
   auto poll = [&]() { return CLUSTER_ACQUIRE ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
@@ -100,7 +101,8 @@ __device__ __forceinline__ bool mbar_wait_thread(uint64_t* bar, uint32_t parity,
   if (!ok) {
     const uint64_t t0 = global_timer_ns();
     for (uint32_t i = 1;; ++i) {
-      if (CLUSTER_ACQUIRE ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait_sleep(bar, parity, 1000u)) {
+      if (CLUSTER_ACQUIRE ? mbar_try_wait_cluster(bar, parity)
+                          : SPIN ? mbar_try_wait(bar, parity) : mbar_try_wait_sleep(bar, parity, 1000u)) {
         ok = true;
         break;
       }
@@ -118,10 +120,10 @@ __device__ __forceinline__ bool mbar_wait_thread(uint64_t* bar, uint32_t parity,
 }
 // The same, called by all 32 lanes of a warp; the result is the same for every lane, so loops
 // that stop on failure stay warp-uniform.
-template <bool CLUSTER_ACQUIRE = false>
+template <bool CLUSTER_ACQUIRE = false, bool SPIN = false>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile uint32_t* abort_word,
                                           uint32_t flag) {
-  return __all_sync(0xFFFFFFFFu, mbar_wait_thread<CLUSTER_ACQUIRE>(bar, parity, abort_word, flag));
+  return __all_sync(0xFFFFFFFFu, mbar_wait_thread<CLUSTER_ACQUIRE, SPIN>(bar, parity, abort_word, flag));
 }
 
 // ---------------------------------------------------------------------------------------

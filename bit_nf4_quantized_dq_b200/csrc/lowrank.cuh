@@ -33,7 +33,12 @@ struct LowRankParams {
   double* partial;        // [splits][cols][rows] float64
 };
 
-constexpr int kLrThreads = 192;
+// Warps: 0 and 6 issue TMA loads (alternate k-blocks), 1 issues MMAs, 2-5 and 7-10 flush to
+// float64 (two groups, each draining half of the columns).
+constexpr int kLrThreads = 352;
+// The accumulator hand-offs between the MMA issuer and the flush warps poll without a
+// suspend hint: each k-block crosses them twice, and a suspended waiter wakes late.
+constexpr bool kLrSpin = true;
 
 template <int BJ, int TERMS>
 struct LrCfg {
@@ -43,9 +48,12 @@ struct LrCfg {
   static constexpr int kBBytes = TERMS * kBTermBytes;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kStagesRaw = (200 * 1024) / kStageBytes;
-  static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
-  static constexpr int kTmemCols = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
-                                   : (2 * BN <= 256) ? 256 : 512;
+  static constexpr int kStages = (kStagesRaw > 8 ? 8 : kStagesRaw) & ~1;   // even: two TMA warps own alternate stages
+  // Accumulator buffers in TMEM: the MMA of k-block it writes buffer it % kBufs while the
+  // flush warps drain older ones; four where they fit in the 512 columns, else two.
+  static constexpr int kBufs = (4 * BN <= 512) ? 4 : 2;
+  static constexpr int kTmemCols = (kBufs * BN <= 32) ? 32 : (kBufs * BN <= 64) ? 64 : (kBufs * BN <= 128) ? 128
+                                   : (kBufs * BN <= 256) ? 256 : 512;
   static constexpr int kSmemBytes = kStages * kStageBytes + 256 + 1024;
   static_assert(BN % 16 == 0 && BN <= 256, "UMMA N");
   static_assert(kBTermBytes % 1024 == 0, "term boxes keep the swizzle atom alignment");
@@ -60,6 +68,21 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16_lr(uint32_t taddr, uint32_t (
       : "r"(taddr));
 }
 
+// One 64-deep k-block into a fresh accumulator: four unrolled 16-deep MMAs whose
+// descriptors differ only in the start address field.
+template <int BN, bool A_MN>
+__device__ __forceinline__ void lr_kblock(uint32_t d, uint32_t a_addr, uint32_t b_addr) {
+  constexpr uint32_t idesc = umma_idesc_bf16(128, BN, A_MN ? 1u : 0u, 0u);
+  const uint64_t a0 = A_MN ? umma_sdesc_sw128(a_addr, 8192u, 1024u) : umma_sdesc_sw128(a_addr, 16u, 1024u);
+  const uint64_t b0 = umma_sdesc_sw128(b_addr, 16u, 1024u);
+#pragma unroll
+  for (int k16 = 0; k16 < 4; ++k16) {
+    const uint64_t ad = a0 + (uint64_t)((A_MN ? 2048u : 32u) * (uint32_t)k16 >> 4);
+    const uint64_t bd = b0 + (uint64_t)(32u * (uint32_t)k16 >> 4);
+    umma_bf16(d, ad, bd, idesc, k16 > 0 ? 1u : 0u);
+  }
+}
+
 template <int BJ, int TERMS>
 __global__ void __launch_bounds__(kLrThreads, 1) lowrank_kernel(const __grid_constant__ LowRankParams p) {
   using C = LrCfg<BJ, TERMS>;
@@ -68,9 +91,10 @@ __global__ void __launch_bounds__(kLrThreads, 1) lowrank_kernel(const __grid_con
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
   uint64_t* empty = full + S;
-  uint64_t* accfull = empty + S;      // [2]
-  uint64_t* accempty = accfull + 2;   // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accempty + 2);
+  constexpr int NB = C::kBufs;
+  uint64_t* accfull = empty + S;      // [NB]
+  uint64_t* accempty = accfull + NB;  // [NB]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accempty + NB);
   volatile uint32_t* abort_word = tmem_slot + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -85,9 +109,9 @@ __global__ void __launch_bounds__(kLrThreads, 1) lowrank_kernel(const __grid_con
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NB; ++b) {
       mbar_init(&accfull[b], 1);
-      mbar_init(&accempty[b], 4);
+      mbar_init(&accempty[b], 8);
     }
     *abort_word = 0u;
     mbar_fence_init();
@@ -105,30 +129,41 @@ __global__ void __launch_bounds__(kLrThreads, 1) lowrank_kernel(const __grid_con
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp == 0) {
+  if (warp == 0 || warp == 6) {
     // ------------------------------------------------------------------ TMA
+    // A bulk-tensor load holds its issuing thread for a few hundred cycles whatever its size,
+    // while loads of different warps, and of different lanes of one instruction, proceed side
+    // by side: two warps take alternate k-blocks, and each k-block's boxes (A, or two halves
+    // of an MN-major A, then one per B term) go out as one instruction from lanes 0..4.
+    const int tw = (warp == 0) ? 0 : 1;
     int last_issue[8];
     for (int s = 0; s < 8; ++s) last_issue[s] = -1;
     bool ok = true;
-    for (int it = 0; it < n_iters; ++it) {
+    for (int it = tw; it < n_iters; it += 2) {
       const int s = it % S;
       const uint32_t ph = (uint32_t)(it / S) & 1u;
       if (!mbar_wait(&empty[s], ph ^ 1u, abort_word, kErrWaitEmpty)) { ok = false; break; }
+      uint8_t* A = smem + s * C::kStageBytes;
+      uint8_t* B = A + C::kABytes;
       if (lane == 0) {
-        uint8_t* A = smem + s * C::kStageBytes;
-        uint8_t* B = A + C::kABytes;
         mbar_arrive_expect_tx(&full[s], C::kABytes + C::kBBytes);
-        const int k = (kb_begin + it) * 64;
-        if (p.a_mn) {
-          tma_load_2d(A, &p.a_map, row0, k, &full[s]);
-          tma_load_2d(A + 8192, &p.a_map, row0 + 64, k, &full[s]);
-        } else {
-          tma_load_2d(A, &p.a_map, k, row0, &full[s]);
-        }
-#pragma unroll
-        for (int t = 0; t < TERMS; ++t) tma_load_2d(B + t * C::kBTermBytes, &p.b_map[t], k, col0, &full[s]);
         last_issue[s] = it;
       }
+      __syncwarp();
+      const int k = (kb_begin + it) * 64;
+      const int na = p.a_mn ? 2 : 1;
+      const CUtensorMap* map = nullptr;
+      uint8_t* dst = nullptr;
+      int cx = 0, cy = 0;
+      if (lane < na) {
+        map = &p.a_map;
+        if (p.a_mn) { dst = A + lane * 8192; cx = row0 + 64 * lane; cy = k; }
+        else { dst = A; cx = k; cy = row0; }
+      } else if (lane < na + TERMS) {
+        const int t = lane - na;
+        map = &p.b_map[t]; dst = B + t * C::kBTermBytes; cx = k; cy = col0;
+      }
+      if (map) tma_load_2d(dst, map, cx, cy, &full[s]);
       __syncwarp();
     }
     if (!ok && lane == 0) {
@@ -141,68 +176,82 @@ __global__ void __launch_bounds__(kLrThreads, 1) lowrank_kernel(const __grid_con
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA
-    const uint32_t idesc = umma_idesc_bf16(128, C::BN, p.a_mn ? 1u : 0u, 0u);
-    for (int it = 0; it < n_iters; ++it) {
-      const int s = it % S;
-      const uint32_t ph = (uint32_t)(it / S) & 1u;
-      const int buf = it & 1;
-      const uint32_t bph = (uint32_t)(it >> 1) & 1u;
-      if (!mbar_wait(&accempty[buf], bph ^ 1u, abort_word, kErrWaitMma)) break;
-      if (!mbar_wait(&full[s], ph, abort_word, kErrWaitTma)) break;
-      tc_fence_after();
-      if (lane == 0) {
+    // Lane 0 alone: the tensor pipe queues only about one MMA ahead, so the issuer keeps
+    // warp-collective instructions out of its loop and issues each k-block unrolled.
+    if (lane == 0) {
+      for (int it = 0; it < n_iters; ++it) {
+        const int s = it % S;
+        const uint32_t ph = (uint32_t)(it / S) & 1u;
+        const int buf = it % NB;
+        const uint32_t bph = (uint32_t)(it / NB) & 1u;
+        if (!mbar_wait_thread<false, kLrSpin>(&accempty[buf], bph ^ 1u, abort_word, kErrWaitMma)) break;
+        if (!mbar_wait_thread(&full[s], ph, abort_word, kErrWaitTma)) break;
+        tc_fence_after();
         const uint32_t a_addr = smem_u32(smem + s * C::kStageBytes);
         const uint32_t b_addr = a_addr + C::kABytes;
-        const int nk16 = (kb_begin + it == p.kblocks - 1) ? p.k16_last : 4;
         const uint32_t d = tmem_base + (uint32_t)(buf * C::BN);
-        for (int k16 = 0; k16 < nk16; ++k16) {
-          const uint64_t ad = p.a_mn ? umma_sdesc_sw128(a_addr + (uint32_t)k16 * 2048u, 8192u, 1024u)
-                                     : umma_sdesc_sw128(a_addr + (uint32_t)k16 * 32u, 16u, 1024u);
-          const uint64_t bd = umma_sdesc_sw128(b_addr + (uint32_t)k16 * 32u, 16u, 1024u);
-          umma_bf16(d, ad, bd, idesc, k16 > 0 ? 1u : 0u);
+        if (kb_begin + it != p.kblocks - 1 || p.k16_last == 4) {
+          if (p.a_mn) lr_kblock<C::BN, true>(d, a_addr, b_addr);
+          else lr_kblock<C::BN, false>(d, a_addr, b_addr);
+        } else {
+          const uint32_t idesc = umma_idesc_bf16(128, C::BN, p.a_mn ? 1u : 0u, 0u);
+          for (int k16 = 0; k16 < p.k16_last; ++k16) {
+            const uint64_t ad = p.a_mn ? umma_sdesc_sw128(a_addr + (uint32_t)k16 * 2048u, 8192u, 1024u)
+                                       : umma_sdesc_sw128(a_addr + (uint32_t)k16 * 32u, 16u, 1024u);
+            const uint64_t bd = umma_sdesc_sw128(b_addr + (uint32_t)k16 * 32u, 16u, 1024u);
+            umma_bf16(d, ad, bd, idesc, k16 > 0 ? 1u : 0u);
+          }
         }
         umma_commit(&empty[s]);
         umma_commit(&accfull[buf]);
       }
-      __syncwarp();
     }
+    __syncwarp();
   } else {
     // ------------------------------------------------------------------ flush to float64
+    // Group g (warps 2-5, then 7-10) drains columns [g * HALF, (g + 1) * HALF) of each
+    // k-block's accumulator; warp w reads TMEM lanes 32 (w % 4) .. 32 (w % 4) + 31.  With
+    // BJ = 16 the second group only keeps the hand-off count.
+    constexpr int HALF = BJ >= 32 ? BJ / 2 : BJ;
+    const int c0 = (warp >= 7) ? HALF : 0;
+    const bool active = c0 < BJ;
     const int q = warp & 3;
     const int row = row0 + 32 * q + lane;
-    double acc[BJ];
+    double acc[HALF];
 #pragma unroll
-    for (int j = 0; j < BJ; ++j) acc[j] = 0.0;
+    for (int j = 0; j < HALF; ++j) acc[j] = 0.0;
     bool ok = true;
     for (int it = 0; it < n_iters; ++it) {
-      const int buf = it & 1;
-      const uint32_t bph = (uint32_t)(it >> 1) & 1u;
-      if (!mbar_wait(&accfull[buf], bph, abort_word, kErrWaitMma)) { ok = false; break; }
+      const int buf = it % NB;
+      const uint32_t bph = (uint32_t)(it / NB) & 1u;
+      if (!mbar_wait<false, kLrSpin>(&accfull[buf], bph, abort_word, kErrWaitMma)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t tb = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * C::BN);
+      if (active) {
+        const uint32_t tb = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * C::BN + c0);
 #pragma unroll
-      for (int j0 = 0; j0 < BJ; j0 += 16) {
-        uint32_t r[TERMS][16];
+        for (int j0 = 0; j0 < HALF; j0 += 16) {
+          uint32_t r[TERMS][16];
 #pragma unroll
-        for (int t = 0; t < TERMS; ++t) tmem_ld_32x32b_x16_lr(tb + (uint32_t)(t * BJ + j0), r[t]);
-        tmem_ld_wait();
+          for (int t = 0; t < TERMS; ++t) tmem_ld_32x32b_x16_lr(tb + (uint32_t)(t * BJ + j0), r[t]);
+          tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          double v = (double)__uint_as_float(r[0][j]);
+          for (int j = 0; j < 16; ++j) {
+            double v = (double)__uint_as_float(r[0][j]);
 #pragma unroll
-          for (int t = 1; t < TERMS; ++t) v += (double)__uint_as_float(r[t][j]);
-          acc[j0 + j] += v;
+            for (int t = 1; t < TERMS; ++t) v += (double)__uint_as_float(r[t][j]);
+            acc[j0 + j] += v;
+          }
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&accempty[buf]);
     }
-    if (ok && row < p.rows) {
+    if (ok && active && row < p.rows) {
       double* out = p.partial + (int64_t)split * p.cols * p.rows;
 #pragma unroll
-      for (int j = 0; j < BJ; ++j) {
-        const int col = col0 + j;
+      for (int j = 0; j < HALF; ++j) {
+        const int col = col0 + c0 + j;
         if (col < p.cols) out[(int64_t)col * p.rows + row] = acc[j];
       }
     }
@@ -267,27 +316,40 @@ __device__ __forceinline__ void split3(double v, uint16_t& a, uint16_t& b, uint1
 // Token-side result (t or u): v = alpha * sum_z partial[z][j][m].  Optional outputs:
 // fp32 [M][r]; bf16 hi / lo [M][r] (two-term split, for the fused GEMMs' adapter k-blocks);
 // the three-term split transposed, T3[term][j][m] with row pitch ldT (for dA / dB).
+// One 32 x 32 tile (m0.., j0..) per block of 32 x 8 threads: the partials are read along m,
+// the [M][r] outputs written along j through a shared-memory transpose.
 __global__ void finalize_tokens_kernel(const double* __restrict__ partial, int splits, int64_t M, int64_t r,
                                        double alpha, float* __restrict__ f32, uint16_t* __restrict__ hi,
                                        uint16_t* __restrict__ lo, uint16_t* __restrict__ T3, int64_t ldT) {
-  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= M * r) return;
-  const int64_t j = idx / M, m = idx % M;
-  double v = 0.0;
-  for (int z = 0; z < splits; ++z) v += partial[((int64_t)z * r + j) * M + m];
-  v *= alpha;
-  if (f32) f32[m * r + j] = (float)v;
-  if (hi) {
-    const __nv_bfloat16 h = __float2bfloat16_rn((float)v);
-    hi[m * r + j] = __bfloat16_as_ushort(h);
-    lo[m * r + j] = bf16_bits_rn(v - (double)__bfloat162float(h));
+  __shared__ double tile[32][33];
+  const int64_t m0 = (int64_t)blockIdx.x * 32, j0 = (int64_t)blockIdx.y * 32;
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int64_t j = j0 + i, m = m0 + threadIdx.x;
+    double v = 0.0;
+    if (m < M && j < r) {
+      for (int z = 0; z < splits; ++z) v += partial[((int64_t)z * r + j) * M + m];
+      v *= alpha;
+      if (T3) {
+        uint16_t a, b, c;
+        split3(v, a, b, c);
+        T3[j * ldT + m] = a;
+        T3[(r + j) * ldT + m] = b;
+        T3[(2 * r + j) * ldT + m] = c;
+      }
+    }
+    tile[i][threadIdx.x] = v;
   }
-  if (T3) {
-    uint16_t a, b, c;
-    split3(v, a, b, c);
-    T3[j * ldT + m] = a;
-    T3[(r + j) * ldT + m] = b;
-    T3[(2 * r + j) * ldT + m] = c;
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int64_t m = m0 + i, j = j0 + threadIdx.x;
+    if (m >= M || j >= r) continue;
+    const double v = tile[threadIdx.x][i];
+    if (f32) f32[m * r + j] = (float)v;
+    if (hi) {
+      const __nv_bfloat16 h = __float2bfloat16_rn((float)v);
+      hi[m * r + j] = __bfloat16_as_ushort(h);
+      lo[m * r + j] = bf16_bits_rn(v - (double)__bfloat162float(h));
+    }
   }
 }
 
@@ -314,25 +376,37 @@ __global__ void split3_T_kernel(const float* __restrict__ t, int64_t M, int64_t 
 }
 
 // Feature-side gradient: g[j][i] = bf16(sum_z partial[z][j][i]); transpose_out = 0 writes
-// out[j * n + i] (dA, [r][K]), 1 writes out[i * r + j] (dB, [N][r]).
+// out[j * n + i] (dA, [r][K]), 1 writes out[i * r + j] (dB, [N][r]).  One 32 x 32 tile
+// (i0.., j0..) per block of 32 x 8 threads; the transposed case goes through shared memory so
+// that both the partials and the output are accessed along their rows.
 __global__ void finalize_grad_kernel(const double* __restrict__ partial, int splits, int64_t r, int64_t n,
                                      uint16_t* __restrict__ out, int transpose_out) {
-  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= r * n) return;
-  int64_t j, i;
-  if (transpose_out) { i = idx / r; j = idx % r; }
-  else { j = idx / n; i = idx % n; }
-  double v = 0.0;
-  for (int z = 0; z < splits; ++z) v += partial[((int64_t)z * r + j) * n + i];
-  out[idx] = bf16_bits_rn(v);
+  __shared__ uint16_t tile[32][34];
+  const int64_t i0 = (int64_t)blockIdx.x * 32, j0 = (int64_t)blockIdx.y * 32;
+  for (int a = threadIdx.y; a < 32; a += blockDim.y) {
+    const int64_t j = j0 + a, i = i0 + threadIdx.x;
+    uint16_t g = 0;
+    if (i < n && j < r) {
+      double v = 0.0;
+      for (int z = 0; z < splits; ++z) v += partial[((int64_t)z * r + j) * n + i];
+      g = bf16_bits_rn(v);
+      if (!transpose_out) out[j * n + i] = g;
+    }
+    tile[a][threadIdx.x] = g;
+  }
+  if (!transpose_out) return;
+  __syncthreads();
+  for (int a = threadIdx.y; a < 32; a += blockDim.y) {
+    const int64_t i = i0 + a, j = j0 + threadIdx.x;
+    if (i < n && j < r) out[i * r + j] = tile[threadIdx.x][a];
+  }
 }
 
 static cudaError_t launch_finalize_tokens(const double* partial, int splits, int64_t M, int64_t r, double alpha,
                                           float* f32, uint16_t* hi, uint16_t* lo, uint16_t* T3, int64_t ldT,
                                           cudaStream_t st) {
-  const int64_t n = M * r;
-  finalize_tokens_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(partial, splits, M, r, alpha, f32, hi, lo,
-                                                                       T3, ldT);
+  dim3 grid((unsigned)((M + 31) / 32), (unsigned)((r + 31) / 32));
+  finalize_tokens_kernel<<<grid, dim3(32, 8), 0, st>>>(partial, splits, M, r, alpha, f32, hi, lo, T3, ldT);
   return cudaGetLastError();
 }
 
@@ -345,8 +419,8 @@ static cudaError_t launch_split3_T(const float* t, int64_t M, int64_t r, uint16_
 
 static cudaError_t launch_finalize_grad(const double* partial, int splits, int64_t r, int64_t n, uint16_t* out,
                                         int transpose_out, cudaStream_t st) {
-  const int64_t total = r * n;
-  finalize_grad_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(partial, splits, r, n, out, transpose_out);
+  dim3 grid((unsigned)((n + 31) / 32), (unsigned)((r + 31) / 32));
+  finalize_grad_kernel<<<grid, dim3(32, 8), 0, st>>>(partial, splits, r, n, out, transpose_out);
   return cudaGetLastError();
 }
 

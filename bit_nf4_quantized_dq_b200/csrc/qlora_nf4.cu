@@ -114,13 +114,23 @@ constexpr int kSms = 148;
 // Split of the K loop over blockIdx.z so that small tile grids still cover the SMs.
 // Every split gets at least one k-block: the count is re-derived from the per-split share.
 int choose_splits(int64_t tiles, int kb) {
+  // Every CTA of these kernels fills an SM (shared memory), so a launch with s splits runs in
+  // ceil(tiles * s / kSms) waves of ceil(kb / s) k-blocks: take the split count with the
+  // fewest k-block steps in total (the smallest on ties), at least 4 k-blocks per split.
   if (tiles >= kSms) return 1;
-  int64_t s = (kSms + tiles - 1) / tiles;
-  const int64_t cap = kb / 4 > 1 ? kb / 4 : 1;
-  if (s > cap) s = cap;
-  if (s < 1) s = 1;
-  const int64_t per = (kb + s - 1) / s;
-  return (int)((kb + per - 1) / per);
+  int best = 1;
+  int64_t best_cost = ((tiles + kSms - 1) / kSms) * (int64_t)kb;
+  const int cap = kb / 4 > 1 ? kb / 4 : 1;
+  for (int s = 2; s <= cap; ++s) {
+    const int64_t per = (kb + s - 1) / s;
+    const int64_t used = (kb + per - 1) / per;   // splits that get k-blocks
+    const int64_t cost = ((tiles * used + kSms - 1) / kSms) * per;
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = (int)used;
+    }
+  }
+  return best;
 }
 
 // ------------------------------------------------------------------------ shapes
