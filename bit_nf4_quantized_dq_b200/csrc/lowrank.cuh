@@ -316,7 +316,7 @@ __device__ __forceinline__ void split3(double v, uint16_t& a, uint16_t& b, uint1
 // Token-side result (t or u): v = alpha * sum_z partial[z][j][m].  Optional outputs:
 // fp32 [M][r]; bf16 hi / lo [M][r] (two-term split, for the fused GEMMs' adapter k-blocks);
 // the three-term split transposed, T3[term][j][m] with row pitch ldT (for dA / dB).
-// One 32 x 32 tile (m0.., j0..) per block of 32 x 8 threads: the partials are read along m,
+// One 32 x 32 tile (m0.., j0..) per block of 32 x 32 threads: the partials are read along m,
 // the [M][r] outputs written along j through a shared-memory transpose.
 __global__ void finalize_tokens_kernel(const double* __restrict__ partial, int splits, int64_t M, int64_t r,
                                        double alpha, float* __restrict__ f32, uint16_t* __restrict__ hi,
@@ -377,7 +377,7 @@ __global__ void split3_T_kernel(const float* __restrict__ t, int64_t M, int64_t 
 
 // Feature-side gradient: g[j][i] = bf16(sum_z partial[z][j][i]); transpose_out = 0 writes
 // out[j * n + i] (dA, [r][K]), 1 writes out[i * r + j] (dB, [N][r]).  One 32 x 32 tile
-// (i0.., j0..) per block of 32 x 8 threads; the transposed case goes through shared memory so
+// (i0.., j0..) per block of 32 x 32 threads; the transposed case goes through shared memory so
 // that both the partials and the output are accessed along their rows.
 __global__ void finalize_grad_kernel(const double* __restrict__ partial, int splits, int64_t r, int64_t n,
                                      uint16_t* __restrict__ out, int transpose_out) {
@@ -406,7 +406,7 @@ static cudaError_t launch_finalize_tokens(const double* partial, int splits, int
                                           float* f32, uint16_t* hi, uint16_t* lo, uint16_t* T3, int64_t ldT,
                                           cudaStream_t st) {
   dim3 grid((unsigned)((M + 31) / 32), (unsigned)((r + 31) / 32));
-  finalize_tokens_kernel<<<grid, dim3(32, 8), 0, st>>>(partial, splits, M, r, alpha, f32, hi, lo, T3, ldT);
+  finalize_tokens_kernel<<<grid, dim3(32, 32), 0, st>>>(partial, splits, M, r, alpha, f32, hi, lo, T3, ldT);
   return cudaGetLastError();
 }
 
@@ -420,7 +420,7 @@ static cudaError_t launch_split3_T(const float* t, int64_t M, int64_t r, uint16_
 static cudaError_t launch_finalize_grad(const double* partial, int splits, int64_t r, int64_t n, uint16_t* out,
                                         int transpose_out, cudaStream_t st) {
   dim3 grid((unsigned)((n + 31) / 32), (unsigned)((r + 31) / 32));
-  finalize_grad_kernel<<<grid, dim3(32, 8), 0, st>>>(partial, splits, r, n, out, transpose_out);
+  finalize_grad_kernel<<<grid, dim3(32, 32), 0, st>>>(partial, splits, r, n, out, transpose_out);
   return cudaGetLastError();
 }
 

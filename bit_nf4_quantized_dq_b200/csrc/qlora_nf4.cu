@@ -115,16 +115,18 @@ constexpr int kSms = 148;
 // Every split gets at least one k-block: the count is re-derived from the per-split share.
 int choose_splits(int64_t tiles, int kb) {
   // Every CTA of these kernels fills an SM (shared memory), so a launch with s splits runs in
-  // ceil(tiles * s / kSms) waves of ceil(kb / s) k-blocks: take the split count with the
-  // fewest k-block steps in total (the smallest on ties), at least 4 k-blocks per split.
+  // ceil(tiles * s / kSms) waves; a wave costs its ceil(kb / s) k-blocks plus a fixed
+  // kSplitOverhead k-blocks' worth of prologue, pipeline fill and partial stores.  Take the
+  // split count with the lowest total (the smallest on ties), at least 4 k-blocks per split.
+  constexpr int64_t kSplitOverhead = 4;
   if (tiles >= kSms) return 1;
   int best = 1;
-  int64_t best_cost = ((tiles + kSms - 1) / kSms) * (int64_t)kb;
+  int64_t best_cost = ((tiles + kSms - 1) / kSms) * ((int64_t)kb + kSplitOverhead);
   const int cap = kb / 4 > 1 ? kb / 4 : 1;
   for (int s = 2; s <= cap; ++s) {
     const int64_t per = (kb + s - 1) / s;
     const int64_t used = (kb + per - 1) / per;   // splits that get k-blocks
-    const int64_t cost = ((tiles * used + kSms - 1) / kSms) * per;
+    const int64_t cost = ((tiles * used + kSms - 1) / kSms) * (per + kSplitOverhead);
     if (cost < best_cost) {
       best_cost = cost;
       best = (int)used;
