@@ -70,6 +70,31 @@ def load_peaks():
 
 
 # ------------------------------------------------------------------------------------------
+# DRAM traffic of the fused GEMMs
+# ------------------------------------------------------------------------------------------
+# Bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum), averaged over the 7 launches
+# of a timed step, from one single-pass capture of this script's own run:
+#   ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum
+#       --clock-control none -k regex:qlora_gemm_kernel -c 42
+#       python bench.py --steps 2 --warmup 1 --no-e2e --no-cpu-baseline
+# They hold only for the kernel sources they were taken on: once any of FUSED_SOURCES changes
+# the traffic is reported as null.
+FUSED_SOURCES = ("gemm.cuh", "gemm.h", "common.cuh", "nf4_device.cuh", "qlora_nf4.cu")
+FUSED_TRAFFIC = {"sources_sha256": "be48b71cc5e3046fc37439a636eab9cf30513ce3931981304f0533d21e3f0bae",
+                 "fwd": 287980233, "dx": 316147694}
+
+
+def fused_traffic(which: str):
+    import hashlib
+    csrc = os.path.join(ROOT, "bit_nf4_quantized_dq_b200", "csrc")
+    h = hashlib.sha256()
+    for f in FUSED_SOURCES:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return FUSED_TRAFFIC[which] if h.hexdigest() == FUSED_TRAFFIC["sources_sha256"] else None
+
+
+# ------------------------------------------------------------------------------------------
 # clocks during the timed region
 # ------------------------------------------------------------------------------------------
 class ClockSampler:
@@ -119,6 +144,68 @@ class ClockSampler:
         os.unlink(self.path)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
                 "reasons": sorted(reasons), "samples": len(sm)}
+
+
+class NvmlClockSampler:
+    """SM clock and clock-event reasons every `period_s` through NVML, in a background thread
+    (nvidia-smi needs over 100 ms before its first sample, longer than a short timed region).
+    The device is found by its PCI bus id; falls back to ClockSampler when NVML is missing."""
+    BITS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20, "sw_power_cap": 0x4}
+
+    def __init__(self, torch_device_index: int, period_s: float = 0.005):
+        self.idx = torch_device_index
+        self.period = period_s
+        self.fallback = None
+        self.samples = []
+        self.thread = None
+        self.stop_flag = None
+
+    def _handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(self.idx)
+        bus = getattr(props, "pci_bus_id", None)
+        if bus is not None:
+            dom = getattr(props, "pci_domain_id", 0)
+            dev = getattr(props, "pci_device_id", 0)
+            return pynvml.nvmlDeviceGetHandleByPciBusId(f"{dom:08x}:{bus:02x}:{dev:02x}.0".encode())
+        return pynvml.nvmlDeviceGetHandleByIndex(self.idx)
+
+    def start(self):
+        import threading
+        try:
+            import pynvml
+            h = self._handle()
+            reasons_fn = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+            self.smax = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.fallback = ClockSampler(self.idx)
+            self.fallback.start()
+            return
+        self.stop_flag = threading.Event()
+
+        def run():
+            while not self.stop_flag.is_set():
+                try:
+                    self.samples.append((pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM), reasons_fn(h)))
+                except Exception:
+                    pass
+                self.stop_flag.wait(self.period)
+
+        self.thread = threading.Thread(target=run, daemon=True)
+        self.thread.start()
+
+    def stop(self) -> dict:
+        if self.fallback is not None:
+            return self.fallback.stop()
+        self.stop_flag.set()
+        self.thread.join(timeout=5)
+        sm = [float(c) for c, _ in self.samples]
+        reasons = sorted({n for _, r in self.samples for n, b in self.BITS.items() if r & b})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": float(self.smax),
+                "reasons": reasons, "samples": len(sm), "source": "nvml"}
 
 
 # ------------------------------------------------------------------------------------------
@@ -244,7 +331,7 @@ def ours(args, rank, world, dev_index):
     # ------------------------------------------------ device-timed run (inputs resident in HBM)
     ev_steps = [make_events(len(bufs)) for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(dev_index)
+    clocks = NvmlClockSampler(dev_index)
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
@@ -297,14 +384,17 @@ def ours(args, rank, world, dev_index):
     # dominant kernel: the fused dequant GEMM with the larger total time
     if acc["fwd_fused"] >= acc["dx_fused"]:
         dom, dom_flops, dom_ms = "fused forward GEMM (NF4 dequant producer + tcgen05)", fused_fwd_flops, acc["fwd_fused"]
+        traffic = fused_traffic("fwd")
     else:
         dom, dom_flops, dom_ms = "fused dX GEMM (NF4 dequant producer + tcgen05)", fused_dx_flops, acc["dx_fused"]
+        traffic = fused_traffic("dx")
     launches_per_linear = [b.plan["fwd_launches"] + b.plan["bwd_launches"] + 4 + 1 for b in bufs]
     achieved = dom_flops / (dom_ms / K) / 1e9
     roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peaks["bf16_tflops_sustained"],
                 "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops_sustained"],
                 "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step)",
-                "traffic": None, "launches_per_step": len(lins), "avg_launch_ms": dom_ms / K / len(lins)}
+                "traffic": traffic, "traffic_unit": "bytes per launch (DRAM read + write, ncu)",
+                "launches_per_step": len(lins), "avg_launch_ms": dom_ms / K / len(lins)}
 
     # ------------------------------------------------ end to end through host buffers
     e2e = None

@@ -21,7 +21,11 @@
 
 namespace qnf4 {
 
-constexpr int kThreads2 = 352;   // TMA warps 0 and 10, MMA warp 1, producer / epilogue warps 2-9
+// TMA warps 0 and 10.. (kTmaWarps2 of them, alternate k-blocks), MMA warp 1, producer / epilogue
+// warps 2-9.  One warp's bulk loads complete one after another, so the ring is spread over
+// several issuing warps.
+constexpr int kTmaWarps2 = 2;
+constexpr int kThreads2 = 320 + 32 * (kTmaWarps2 - 1);
 
 struct Cfg2 {
   static constexpr int BN = 256;                    // UMMA N (tokens per pair)
@@ -39,6 +43,7 @@ struct Cfg2 {
   //    most one phase behind the phase it waits for.
   static_assert(kTStages % 2 == 0 && kASlots % 2 == 0, "rings must split evenly between the producer groups");
   static_assert(kTStages <= 2 * kASlots, "TMA run-ahead must not alias the A-slot barrier phases");
+  static_assert(kTStages % kTmaWarps2 == 0 && kASlots % kTmaWarps2 == 0, "each TMA warp owns whole stages and A slots");
   static constexpr int kBarrierOffset = kTStages * kTStageBytes + kASlots * kABytes;
   static constexpr int kTmemCols = 256;
   static constexpr int kSmemBytes = kBarrierOffset + 512 + 1024;   // rings, barriers, alignment
@@ -182,17 +187,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
 
   if (warp == 0 || warp >= 10) {
     // ------------------------------------------------------------------ TMA (both CTAs)
-    // Two warps (0 and 10) take alternate k-blocks: a bulk-tensor load holds its issuing
+    // kTmaWarps2 warps (0, 10, ..) take turns on k-blocks: a bulk-tensor load holds its issuing
     // thread for a few hundred cycles whatever its size, while loads of different warps, and
     // of different lanes of one instruction, proceed side by side.  Each k-block's loads go
     // out as one instruction: lane 0 this CTA's half of the B tile, lane 1 the codes (or the
     // A tile), lane 2 the second half of an MN-major A tile.  All use the pair form, which
     // completes on any mbarrier of the pair: the even CTA's full[s], or this CTA's cfull[s].
-    const int tw = (warp == 0) ? 0 : 1;
+    const int tw = (warp == 0) ? 0 : warp - 9;
     int last_issue[ST];
     for (int s = 0; s < ST; ++s) last_issue[s] = -1;
     bool ok = true;
-    for (int it = tw; it < n_iters && ok; it += 2) {
+    for (int it = tw; it < n_iters && ok; it += kTmaWarps2) {
       const int s = it % ST, a = it % SA;
       const uint32_t ph = (uint32_t)(it / ST) & 1u, pa = (uint32_t)(it / SA) & 1u;
       if (!mbar_wait(&empty[s], ph ^ 1u, abort_word, kErrWaitEmpty)) { ok = false; break; }
