@@ -34,9 +34,13 @@ constexpr int kTmaWarps = 2;
 constexpr int kThreads = 320 + 32 * (kTmaWarps - 1);   // + MMA warp, two groups of four producer / epilogue warps
 constexpr int kCodesBytes = 4096;   // packed codes of one 128 x 64 weight tile
 
-template <int BN>
+// A_TMEM: the A tile lives in tensor memory (slot s at column kATmemCol0 + 32 s), so a stage
+// holds only B and the codes and more stages fit.
+constexpr uint32_t kATmemCol0 = 256;
+
+template <int BN, bool A_TMEM = false>
 struct Cfg {
-  static constexpr int kABytes = kBM * kBK * 2;
+  static constexpr int kABytes = A_TMEM ? 0 : kBM * kBK * 2;
   static constexpr int kBBytes = BN * kBK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes + kCodesBytes;
   static constexpr int kStagesRaw = (220 * 1024 - 2048) / kStageBytes;
@@ -44,7 +48,8 @@ struct Cfg {
   // stages and wait on every phase of their barriers (a parity wait that skips a phase can
   // pass early).
   static constexpr int kStages = (kStagesRaw > 8 ? 8 : kStagesRaw) & ~1;
-  static constexpr int kTmemCols = BN <= 32 ? 32 : BN;
+  static constexpr int kTmemCols = A_TMEM ? 512 : (BN <= 32 ? 32 : BN);
+  static_assert(!A_TMEM || (BN == 256 && kStages <= 8), "A in TMEM: 256-column accumulator + 8 slots of 32 columns");
   static constexpr int kBarrierBytes = 256;
   static constexpr int kSmemBytes = kStages * kStageBytes + kBarrierBytes + 1024;
   static_assert(kStages >= 2 && kStages % 2 == 0, "pipeline too shallow, or odd");
@@ -143,6 +148,50 @@ __device__ __forceinline__ UnitScale fetch_scale(const GemmParams& p, const Unit
   return r;
 }
 
+// tcgen05.mma with the A operand in tensor memory (kind::f16, bf16 x bf16 -> fp32): row i of A
+// is TMEM lane i, two consecutive K elements per 32-bit column.
+__device__ __forceinline__ void umma_bf16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 32 consecutive 32-bit columns of this warp's 32 TMEM lanes (one lane per thread).
+__device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+      "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
+      "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
+      "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// One k-block with A in TMEM: four 16-deep MMAs, A advancing 8 columns per slice.
+template <int BN>
+__device__ __forceinline__ void umma_kblock_ts(uint32_t tmem_acc, uint32_t a_tmem, uint32_t b_addr, uint32_t acc,
+                                               int nk16) {
+  constexpr uint32_t idesc = umma_idesc_bf16(kBM, BN, 0u, 0u);
+  const uint64_t b0 = umma_sdesc_sw128(b_addr, 16u, 1024u);
+  if (nk16 == 4) {
+#pragma unroll
+    for (int k16 = 0; k16 < 4; ++k16)
+      umma_bf16_ts(tmem_acc, a_tmem + 8u * (uint32_t)k16, b0 + (uint64_t)(32u * (uint32_t)k16 >> 4), idesc,
+                   k16 == 0 ? acc : 1u);
+  } else {
+    for (int k16 = 0; k16 < nk16; ++k16)
+      umma_bf16_ts(tmem_acc, a_tmem + 8u * (uint32_t)k16, b0 + (uint64_t)(32u * (uint32_t)k16 >> 4), idesc,
+                   (acc || k16 > 0) ? 1u : 0u);
+  }
+}
+
 // One k-block (64 deep) of MMAs: four 16-deep tcgen05.mma into the accumulator.  The
 // descriptors of consecutive 16-deep slices differ only in their start address (bits 0-13,
 // 16-byte units): 32 bytes along a K-major row, 2048 bytes (16 K rows of 128 bytes) down an
@@ -173,9 +222,9 @@ __device__ __noinline__ void umma_kblock_ragged(uint32_t tmem_acc, uint32_t a_ad
   }
 }
 
-template <int BN, bool GENERIC>
+template <int BN, bool GENERIC, bool A_TMEM>
 __global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_constant__ GemmParams p) {
-  using C = Cfg<BN>;
+  using C = Cfg<BN, A_TMEM>;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_dyn[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
@@ -258,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_co
         } else if (sg.a_src == kANf4MN) {
           if (!GENERIC) { map = sg.a_map; dst = stage_c(s); cx = row0 / 2; cy = k; }
         } else if (sg.a_src == kATmaK) {
-          map = sg.a_map; dst = stage_a(s); cx = k; cy = row0;
+          if (!A_TMEM) { map = sg.a_map; dst = stage_a(s); cx = k; cy = row0; }
         } else {
           map = sg.a_map; dst = stage_a(s); cx = row0; cy = k;
         }
@@ -299,7 +348,11 @@ __global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_co
         const uint32_t a_addr = smem_u32(stage_a(s));
         const uint32_t b_addr = smem_u32(stage_b(s));
         const uint32_t acc = it > 0 ? 1u : 0u;
-        if (!ip.last || sg.k16_last == 4) {
+        if constexpr (A_TMEM) {
+          (void)a_mn; (void)a_addr;
+          umma_kblock_ts<BN>(tmem_acc, tmem_acc + kATmemCol0 + 32u * (uint32_t)s, b_addr, acc,
+                             ip.last ? sg.k16_last : 4);
+        } else if (!ip.last || sg.k16_last == 4) {
           if (a_mn) umma_kblock<BN, true>(tmem_acc, a_addr, b_addr, acc);
           else umma_kblock<BN, false>(tmem_acc, a_addr, b_addr, acc);
         } else {
@@ -315,7 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_co
     // Two groups of four warps take alternate k-blocks; within a group thread t owns one
     // 64-weight unit per k-block.
     const int grp = (warp - 2) >> 2;          // 0: warps 2-5, 1: warps 6-9
-    const int t = (threadIdx.x - 64) & 127;
+    const int t = 32 * (warp & 3) + lane;       // tile row t = TMEM lane t (warp w reaches lanes 32 (w % 4) ..)
     bool ok = true;
     if (p.has_nf4) {
       const float mean = __ldg(p.mean);
@@ -355,7 +408,40 @@ __global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_co
           }
         }
         if (!mbar_wait(&full[s], ph, abort_word, kErrWaitTma)) { ok = false; break; }
-        if (nf4) {
+        if constexpr (A_TMEM) {
+          // Row t of the A tile (64 bf16 = 32 columns) into TMEM slot s.  Slot s is free: full[s]
+          // of this iteration follows the release of stage s by the MMAs that last read it.
+          uint32_t v[32];
+          if (nf4) {
+            if constexpr (!GENERIC) {
+              const uint4* src = reinterpret_cast<const uint4*>(stage_c(s) + t * 32);
+              const uint4 c0 = src[0], c1 = src[1];
+              words[0] = c0.x; words[1] = c0.y; words[2] = c0.z; words[3] = c0.w;
+              words[4] = c1.x; words[5] = c1.y; words[6] = c1.z; words[7] = c1.w;
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              uint32_t o[4] = {0u, 0u, 0u, 0u};
+              if (!GENERIC || j < sc.valid) nf4_expand8(words[j], (GENERIC && j >= sc.split) ? L1 : L0, o);
+              v[4 * j] = o[0]; v[4 * j + 1] = o[1]; v[4 * j + 2] = o[2]; v[4 * j + 3] = o[3];
+            }
+          } else {
+            // a kATmaK stretch: row t of the adapter matrix, k-block kb, from global memory
+            const IterPos ip = iter_pos(p, it, kb_begin, kb_end, first_split);
+            const int64_t row = (int64_t)row0 + t;
+            const int64_t kk = (int64_t)p.seg[ip.seg].a_k0 + (int64_t)ip.kb * kBK;
+            const uint4* src = reinterpret_cast<const uint4*>(p.a_glob + row * p.a_glob_ld + kk);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              uint4 w4 = make_uint4(0u, 0u, 0u, 0u);
+              if (row < p.a_glob_rows && kk + 8 * q + 8 <= p.a_glob_cols) w4 = __ldg(src + q);
+              v[4 * q] = w4.x; v[4 * q + 1] = w4.y; v[4 * q + 2] = w4.z; v[4 * q + 3] = w4.w;
+            }
+          }
+          tmem_st_32x32b_x32(tmem_acc + ((uint32_t)(32 * (warp & 3)) << 16) + kATmemCol0 + 32u * (uint32_t)s, v);
+          tmem_st_wait();
+          tc_fence_before();
+        } else if (nf4) {
           uint8_t* A = stage_a(s);
           if constexpr (!GENERIC) {
             const uint4* src = reinterpret_cast<const uint4*>(stage_c(s) + t * 32);
@@ -427,24 +513,28 @@ __global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_co
   }
 }
 
-template <int BN, bool GENERIC>
+template <int BN, bool GENERIC, bool A_TMEM = false>
 static cudaError_t launch_bn(const GemmParams& p, cudaStream_t st) {
-  using C = Cfg<BN>;
+  using C = Cfg<BN, A_TMEM>;
   static bool configured = false;   // per process; the attribute is per function, not per device
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(qlora_gemm_kernel<BN, GENERIC>,
+    cudaError_t e = cudaFuncSetAttribute(qlora_gemm_kernel<BN, GENERIC, A_TMEM>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     configured = true;
   }
   dim3 grid((p.rows + kBM - 1) / kBM, (p.cols + BN - 1) / BN, p.splits);
-  qlora_gemm_kernel<BN, GENERIC><<<grid, kThreads, C::kSmemBytes, st>>>(p);
+  qlora_gemm_kernel<BN, GENERIC, A_TMEM><<<grid, kThreads, C::kSmemBytes, st>>>(p);
   return cudaGetLastError();
 }
 
 template <bool GENERIC>
 static cudaError_t launch_gemm_g(const GemmParams& p, int bn, cudaStream_t st) {
   if (p.b_box_rows != bn) return cudaErrorInvalidValue;   // each B box must fill exactly one B tile
+  if (p.a_tmem) {                                         // A in tensor memory: 256-token tiles only
+    if (bn != 256) return cudaErrorInvalidValue;
+    return launch_bn<256, GENERIC, true>(p, st);
+  }
   switch (bn) {
     case 16: return launch_bn<16, GENERIC>(p, st);
     case 32: return launch_bn<32, GENERIC>(p, st);

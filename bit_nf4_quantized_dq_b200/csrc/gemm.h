@@ -42,6 +42,12 @@ struct GemmParams {
   int32_t splits, kb_per_split;  // segment 0 is split over blockIdx.z; later segments run in split 0
   int32_t has_nf4, nf4_generic;  // NF4 producer present; codes fetched without TMA (K % 64 != 0)
   int32_t b_box_rows;            // rows of every B-operand TMA box (checked against the kernel's tile)
+  // A operand in tensor memory (forward, 256-token tiles): the producers write the dequantized
+  // tile, and the rows of kATmaK stretches from a_glob ([a_glob_rows][a_glob_cols] bf16, row
+  // pitch a_glob_ld elements), straight into TMEM; shared memory holds only B and the codes.
+  int32_t a_tmem;
+  const uint16_t* a_glob;
+  int64_t a_glob_ld, a_glob_rows, a_glob_cols;
   // NF4 operand: codes / scale codes / group constants / mean of W [nw][kw]
   const uint8_t* codes;
   const uint8_t* scale_codes;

@@ -277,6 +277,8 @@ int run_lowrank(const void* a_base, bool a_mn, int64_t a_inner, int64_t a_outer,
 // (cta_group::2, gemm2sm.cuh).  Rows of each B-operand TMA box: a CTA of a pair loads half of
 // the 256-token tile.
 constexpr bool kPairTiles = false;
+// The fused forward keeps its A operand in tensor memory (gemm.cuh, A_TMEM) on 256-token tiles.
+constexpr bool kATmemForward = true;
 int b_box_rows(int bn) { return (kPairTiles && bn == 256) ? 128 : bn; }
 
 cudaError_t launch_fused(const qnf4::GemmParams& gp, int bn, cudaStream_t st) {
@@ -492,6 +494,15 @@ int qlora_linear_fwd(const uint16_t* x, int64_t M, int64_t K, int64_t N, const u
     gp.seg[0] = qnf4::GemmSeg{kblocks(K), k16_last(K), qnf4::kANf4K, 0, 1, 0, 0, 0};
     gp.seg[1] = qnf4::GemmSeg{kblocks(r), k16_last(r), qnf4::kATmaK, 2, 3, 0, 0, 0};
     gp.seg[2] = qnf4::GemmSeg{kblocks(r), k16_last(r), qnf4::kATmaK, 2, 4, 0, 0, 0};
+    if (kATmemForward && plan.bn == 256 && !kPairTiles) {
+      // 256-token tiles keep the dequantized W tile (and the adapter matrix rows) in tensor
+      // memory, which leaves shared memory for 6 stages instead of 4
+      gp.a_tmem = 1;
+      gp.a_glob = B;
+      gp.a_glob_ld = r;
+      gp.a_glob_rows = N;
+      gp.a_glob_cols = r;
+    }
     gp.rows = (int32_t)N;
     gp.cols = (int32_t)M;
     gp.splits = plan.splits;
