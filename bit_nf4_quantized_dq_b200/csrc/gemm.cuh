@@ -100,6 +100,7 @@ struct UnitGeom {
   int64_t kcol;   // first W column of the unit
   uint32_t dst;   // byte offset of the unit's 128-byte row inside the A tile
   uint32_t swz;   // row & 7
+  uint32_t coff;  // byte offset of the unit's 32 code bytes inside the stage's codes tile
 };
 
 __device__ __forceinline__ UnitGeom unit_geom(int a_src, int t, int row0, int64_t k) {
@@ -109,12 +110,18 @@ __device__ __forceinline__ UnitGeom unit_geom(int a_src, int t, int row0, int64_
     u.kcol = k;
     u.dst = (uint32_t)t * 128u;
     u.swz = (uint32_t)t & 7u;
+    u.coff = (uint32_t)t * 32u;     // codes tile [128 W rows][32 bytes]
   } else {                          // dX: columns row0.. of W, k-block k of its rows
-    const int nl = t >> 1, half = t & 1;
+    // Thread t = 8 g + l takes W row nl = 8 (g / 2) + l and column half ((l / 2) & 1) ^ (g & 1):
+    // every 8 lanes then write 8 different rows (their swizzled 16-byte chunks never share a
+    // bank), and their code loads (codes tile [64 W rows][64 bytes]) meet at most 2-way.
+    const int g = t >> 3, l = t & 7;
+    const int nl = 8 * (g >> 1) + l, half = ((l >> 1) & 1) ^ (g & 1);
     u.n = k + nl;
     u.kcol = (int64_t)row0 + 64 * half;
     u.dst = (uint32_t)half * 8192u + (uint32_t)nl * 128u;
     u.swz = (uint32_t)nl & 7u;
+    u.coff = (uint32_t)nl * 64u + (uint32_t)half * 32u;
   }
   return u;
 }
@@ -414,7 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_co
           uint32_t v[32];
           if (nf4) {
             if constexpr (!GENERIC) {
-              const uint4* src = reinterpret_cast<const uint4*>(stage_c(s) + t * 32);
+              const uint4* src = reinterpret_cast<const uint4*>(stage_c(s) + u.coff);
               const uint4 c0 = src[0], c1 = src[1];
               words[0] = c0.x; words[1] = c0.y; words[2] = c0.z; words[3] = c0.w;
               words[4] = c1.x; words[5] = c1.y; words[6] = c1.z; words[7] = c1.w;
@@ -444,7 +451,7 @@ __global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_co
         } else if (nf4) {
           uint8_t* A = stage_a(s);
           if constexpr (!GENERIC) {
-            const uint4* src = reinterpret_cast<const uint4*>(stage_c(s) + t * 32);
+            const uint4* src = reinterpret_cast<const uint4*>(stage_c(s) + u.coff);
             const uint4 c0 = src[0], c1 = src[1];
             words[0] = c0.x; words[1] = c0.y; words[2] = c0.z; words[3] = c0.w;
             words[4] = c1.x; words[5] = c1.y; words[6] = c1.z; words[7] = c1.w;

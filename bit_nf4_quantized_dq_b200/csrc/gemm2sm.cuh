@@ -332,7 +332,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
       if (nf4) {
         uint8_t* A = aslot(a);
         if constexpr (!GENERIC) {
-          const uint4* src = reinterpret_cast<const uint4*>(tstage_c(s) + t * 32);
+          const uint4* src = reinterpret_cast<const uint4*>(tstage_c(s) + u.coff);
           const uint4 c0 = src[0], c1 = src[1];
           words[0] = c0.x; words[1] = c0.y; words[2] = c0.z; words[3] = c0.w;
           words[4] = c1.x; words[5] = c1.y; words[6] = c1.z; words[7] = c1.w;
