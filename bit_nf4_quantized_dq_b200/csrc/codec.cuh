@@ -28,22 +28,24 @@ struct BucketEntry {
   float thr;
 };
 
+// Thread b < 33 computes bucket b once and fills its 32 per-lane copies (one copy per lane
+// keeps the lookups of a warp free of bank conflicts).
 __device__ __forceinline__ void build_bucket_table(BucketEntry (*tab)[32]) {
   constexpr float q[16] = QNF4_LEVELS;
-  for (int i = threadIdx.x; i < 33 * 32; i += blockDim.x) {
-    const int b = i / 32;
-    // bucket b holds the fp32 n with round(16 n + 16) == b
-    const double lo = (b - 16.5) / 16.0, hi = (b - 15.5) / 16.0;
-    uint32_t base = 0;
-    float thr = __int_as_float(0x7F800000);  // +inf: no midpoint inside
-    for (int j = 0; j < 15; ++j) {
-      const double m = 0.5 * ((double)q[j] + (double)q[j + 1]);   // exact in float64
-      const float theta = __double2float_rd(m);
-      if ((double)theta < lo) ++base;
-      else if ((double)theta < hi) thr = theta;
-    }
-    tab[b][i % 32] = BucketEntry{base, thr};
+  const int b = threadIdx.x;
+  if (b >= 33) return;
+  // bucket b holds the fp32 n with round(16 n + 16) == b
+  const double lo = (b - 16.5) / 16.0, hi = (b - 15.5) / 16.0;
+  uint32_t base = 0;
+  float thr = __int_as_float(0x7F800000);  // +inf: no midpoint inside
+  for (int j = 0; j < 15; ++j) {
+    const double m = 0.5 * ((double)q[j] + (double)q[j + 1]);   // exact in float64
+    const float theta = __double2float_rd(m);
+    if ((double)theta < lo) ++base;
+    else if ((double)theta < hi) thr = theta;
   }
+  const BucketEntry e{base, thr};
+  for (int l = 0; l < 32; ++l) tab[b][l] = e;
 }
 
 __device__ __forceinline__ uint32_t nearest_code(float n, const BucketEntry (*tab)[32], int lane) {
