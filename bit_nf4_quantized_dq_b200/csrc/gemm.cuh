@@ -50,7 +50,7 @@ struct Cfg {
   static constexpr int kStages = (kStagesRaw > 8 ? 8 : kStagesRaw) & ~1;
   static constexpr int kTmemCols = A_TMEM ? 512 : (BN <= 32 ? 32 : BN);
   static_assert(!A_TMEM || (BN == 256 && kStages <= 8), "A in TMEM: 256-column accumulator + 8 slots of 32 columns");
-  static constexpr int kBarrierBytes = 256;
+  static constexpr int kBarrierBytes = 512;
   static constexpr int kSmemBytes = kStages * kStageBytes + kBarrierBytes + 1024;
   static_assert(kStages >= 2 && kStages % 2 == 0, "pipeline too shallow, or odd");
   static_assert(kStages % kTmaWarps == 0, "each TMA warp must own whole stages");
@@ -236,7 +236,8 @@ __global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_co
   extern __shared__ uint8_t smem_dyn[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
-  uint64_t* prod = full + S;
+  uint64_t* cfull = full + S;   // the stage's codes have landed (or a plain arrive): producers may start
+  uint64_t* prod = cfull + S;
   uint64_t* empty = prod + S;
   uint64_t* accfull = empty + S;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accfull + 1);
@@ -255,6 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_co
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
+      mbar_init(&cfull[s], 1);
       mbar_init(&prod[s], 4);
       mbar_init(&empty[s], 1);
     }
@@ -290,12 +292,13 @@ __global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_co
       if (!mbar_wait(&empty[s], ph ^ 1u, abort_word, kErrWaitEmpty)) { ok = false; break; }
       const IterPos ip = iter_pos(p, it, kb_begin, kb_end, first_split);
       const GemmSeg& sg = p.seg[ip.seg];
+      const bool nf4 = (sg.a_src == kANf4K || sg.a_src == kANf4MN);
       if (lane == 0) {
-        uint32_t bytes = C::kBBytes;
-        const bool nf4 = (sg.a_src == kANf4K || sg.a_src == kANf4MN);
-        if (nf4 && !GENERIC) bytes += kCodesBytes;
-        if (!nf4) bytes += C::kABytes;
-        mbar_arrive_expect_tx(&full[s], bytes);
+        // The codes complete on cfull[s], so the producers can dequantize while the (larger)
+        // B tile is still landing on full[s].
+        mbar_arrive_expect_tx(&full[s], C::kBBytes + (nf4 ? 0u : (uint32_t)C::kABytes));
+        if (nf4 && !GENERIC) mbar_arrive_expect_tx(&cfull[s], kCodesBytes);
+        else mbar_arrive(&cfull[s]);
         last_issue[s] = it;
       }
       __syncwarp();
@@ -306,13 +309,14 @@ __global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_co
       const int k = sg.a_k0 + ip.kb * kBK;
       int map = -1, cx = 0, cy = 0;
       uint8_t* dst = nullptr;
+      uint64_t* bar = &full[s];
       if (lane == 0) {
         map = sg.b_map; dst = stage_b(s); cx = sg.b_k0 + ip.kb * kBK; cy = col0;
       } else if (lane == 1) {
         if (sg.a_src == kANf4K) {
-          if (!GENERIC) { map = sg.a_map; dst = stage_c(s); cx = k / 2; cy = row0; }
+          if (!GENERIC) { map = sg.a_map; dst = stage_c(s); cx = k / 2; cy = row0; bar = &cfull[s]; }
         } else if (sg.a_src == kANf4MN) {
-          if (!GENERIC) { map = sg.a_map; dst = stage_c(s); cx = row0 / 2; cy = k; }
+          if (!GENERIC) { map = sg.a_map; dst = stage_c(s); cx = row0 / 2; cy = k; bar = &cfull[s]; }
         } else if (sg.a_src == kATmaK) {
           if (!A_TMEM) { map = sg.a_map; dst = stage_a(s); cx = k; cy = row0; }
         } else {
@@ -321,7 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_co
       } else if (lane == 2 && sg.a_src == kATmaMN) {
         map = sg.a_map; dst = stage_a(s) + 8192; cx = row0 + 64; cy = k;
       }
-      if (map >= 0) tma_load_2d(dst, &p.maps[map], cx, cy, &full[s]);
+      if (map >= 0) tma_load_2d(dst, &p.maps[map], cx, cy, bar);
       __syncwarp();
     }
     if (!ok && lane == 0) {
@@ -330,6 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_co
         if (last_issue[s] >= 0) {
           const uint32_t ph = (uint32_t)(last_issue[s] / S) & 1u;
           for (int i = 0; i < (1 << 20) && !mbar_try_wait(&full[s], ph); ++i) {}
+          for (int i = 0; i < (1 << 20) && !mbar_try_wait(&cfull[s], ph); ++i) {}
         }
     }
     __syncwarp();
@@ -414,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_co
             for (int j = 0; j < 8; ++j) words[j] = (j < sc.valid) ? __ldg(src + j) : 0u;
           }
         }
-        if (!mbar_wait(&full[s], ph, abort_word, kErrWaitTma)) { ok = false; break; }
+        if (!mbar_wait(&cfull[s], ph, abort_word, kErrWaitTma)) { ok = false; break; }
         if constexpr (A_TMEM) {
           // Row t of the A tile (64 bf16 = 32 columns) into TMEM slot s.  Slot s is free: full[s]
           // of this iteration follows the release of stage s by the MMAs that last read it.
@@ -471,6 +476,8 @@ __global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_co
           }
           fence_proxy_async_smem();
         }
+        // prod[s] is the MMA issuer's only wait, so it also vouches for the B tile
+        if (!mbar_wait(&full[s], ph, abort_word, kErrWaitTma)) { ok = false; break; }
         __syncwarp();
         if (lane == 0) mbar_arrive(&prod[s]);
       }
