@@ -10,9 +10,9 @@
 //
 // The tensor cores multiply exact bf16 values (x, dY, A, B, or an exact three-term bf16
 // split of an fp32 t or u: fp32 = t1 + t2 + t3 with 8 significant bits each) and accumulate
-// one 64-wide k-block at a time in TMEM (fp32).  After every k-block the epilogue warps move
-// the block sums into float64 registers (TMEM is double-buffered so the next k-block's MMAs
-// overlap the flush), adding the three split terms of a column in float64.  The float64
+// one 64-wide k-block at a time in TMEM (fp32).  After every k-block eight flush warps move
+// the block sums into float64 registers (up to four TMEM accumulator buffers, so the next
+// k-blocks' MMAs overlap the flush), adding the three split terms of a column in float64.  The float64
 // partial of each K split goes to the workspace; a finalize kernel sums the splits.  With
 // the long reductions here (thousands of tokens), plain fp32 accumulation leaves errors far
 // above the elementwise absolute floor at outputs that cancel to near zero; this keeps the

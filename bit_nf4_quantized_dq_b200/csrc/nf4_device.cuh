@@ -107,20 +107,4 @@ __device__ __forceinline__ void nf4_expand8(uint32_t w, const Nf4Lut& L, uint32_
   }
 }
 
-// Expansion where each element chooses between two tables (a block boundary inside the
-// eight elements): element i uses `B` when i >= split, else `A`.
-__device__ __forceinline__ void nf4_expand8_two(uint32_t w, const Nf4Lut& A, const Nf4Lut& B, int split,
-                                                uint32_t (&o)[4]) {
-  uint32_t oa[4], ob[4];
-  nf4_expand8(w, A, oa);
-  nf4_expand8(w, B, ob);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint32_t lo_b = (2 * i >= split) ? 0x0000FFFFu : 0u;
-    const uint32_t hi_b = (2 * i + 1 >= split) ? 0xFFFF0000u : 0u;
-    const uint32_t mb = lo_b | hi_b;
-    o[i] = (oa[i] & ~mb) | (ob[i] & mb);
-  }
-}
-
 }  // namespace qnf4
