@@ -294,10 +294,13 @@ __global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_co
       const GemmSeg& sg = p.seg[ip.seg];
       const bool nf4 = (sg.a_src == kANf4K || sg.a_src == kANf4MN);
       if (lane == 0) {
-        // The codes complete on cfull[s], so the producers can dequantize while the (larger)
-        // B tile is still landing on full[s].
-        mbar_arrive_expect_tx(&full[s], C::kBBytes + (nf4 ? 0u : (uint32_t)C::kABytes));
-        if (nf4 && !GENERIC) mbar_arrive_expect_tx(&cfull[s], kCodesBytes);
+        // With A in shared memory the codes complete on cfull[s], so the producers can
+        // dequantize while the (larger) B tile is still landing on full[s].  With A in tensor
+        // memory (6 stages) that gains nothing and the codes complete on full[s].
+        const bool codes_tma = nf4 && !GENERIC;
+        mbar_arrive_expect_tx(&full[s], C::kBBytes + (nf4 ? 0u : (uint32_t)C::kABytes) +
+                                            ((A_TMEM && codes_tma) ? (uint32_t)kCodesBytes : 0u));
+        if (!A_TMEM && codes_tma) mbar_arrive_expect_tx(&cfull[s], kCodesBytes);
         else mbar_arrive(&cfull[s]);
         last_issue[s] = it;
       }
@@ -314,9 +317,9 @@ __global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_co
         map = sg.b_map; dst = stage_b(s); cx = sg.b_k0 + ip.kb * kBK; cy = col0;
       } else if (lane == 1) {
         if (sg.a_src == kANf4K) {
-          if (!GENERIC) { map = sg.a_map; dst = stage_c(s); cx = k / 2; cy = row0; bar = &cfull[s]; }
+          if (!GENERIC) { map = sg.a_map; dst = stage_c(s); cx = k / 2; cy = row0; bar = A_TMEM ? &full[s] : &cfull[s]; }
         } else if (sg.a_src == kANf4MN) {
-          if (!GENERIC) { map = sg.a_map; dst = stage_c(s); cx = row0 / 2; cy = k; bar = &cfull[s]; }
+          if (!GENERIC) { map = sg.a_map; dst = stage_c(s); cx = row0 / 2; cy = k; bar = A_TMEM ? &full[s] : &cfull[s]; }
         } else if (sg.a_src == kATmaK) {
           if (!A_TMEM) { map = sg.a_map; dst = stage_a(s); cx = k; cy = row0; }
         } else {
@@ -419,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_co
             for (int j = 0; j < 8; ++j) words[j] = (j < sc.valid) ? __ldg(src + j) : 0u;
           }
         }
-        if (!mbar_wait(&cfull[s], ph, abort_word, kErrWaitTma)) { ok = false; break; }
+        if (!mbar_wait(A_TMEM ? &full[s] : &cfull[s], ph, abort_word, kErrWaitTma)) { ok = false; break; }
         if constexpr (A_TMEM) {
           // Row t of the A tile (64 bf16 = 32 columns) into TMEM slot s.  Slot s is free: full[s]
           // of this iteration follows the release of stage s by the MMAs that last read it.
@@ -477,7 +480,7 @@ __global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_co
           fence_proxy_async_smem();
         }
         // prod[s] is the MMA issuer's only wait, so it also vouches for the B tile
-        if (!mbar_wait(&full[s], ph, abort_word, kErrWaitTma)) { ok = false; break; }
+        if (!A_TMEM && !mbar_wait(&full[s], ph, abort_word, kErrWaitTma)) { ok = false; break; }
         __syncwarp();
         if (lane == 0) mbar_arrive(&prod[s]);
       }
