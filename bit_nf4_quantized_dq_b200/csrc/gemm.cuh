@@ -1,23 +1,28 @@
 // tcgen05 GEMM engine with an on-chip NF4 -> bf16 dequant producer.
 //
 // D[rows x cols] (fp32, in TMEM) = sum over K-loop stretches of A[rows x k] * B[cols x k]^T.
-// The 128-row A side is either loaded by TMA or produced on chip from packed NF4 codes (the
-// dequantized 16-bit weights exist only in shared memory, never in HBM); the B side is a
-// K-major bf16 tile loaded by TMA.  One elected thread issues tcgen05.mma (kind::f16,
-// bf16 x bf16 -> fp32) into a TMEM accumulator; four warps read it back for the epilogue.
+// The 128-row A side is either loaded by TMA or produced on chip from packed NF4 codes; the
+// dequantized 16-bit weights exist only in shared memory or, with A_TMEM, in tensor memory,
+// never in HBM.  The B side is a K-major bf16 tile loaded by TMA.  Lane 0 of warp 1 issues
+// tcgen05.mma (kind::f16, bf16 x bf16 -> fp32) into the TMEM accumulator; the eight producer
+// warps read it back for the epilogue.
 //
 // The method's forward and backward ("QLoRA Paper Breakdown: 4-Bit NormalFloat (NF4), Double
-// Quantization, and Paged Optimizers" (fullstackaihub), section 4) map onto this engine as
+// Quantization, and Paged Optimizers" (fullstackaihub), section 4) use this engine for
 //   y^T  = W' x^T + B t^T            (rows = out features, cols = tokens)
 //   dX^T = W'^T dY^T + A^T u^T       (rows = in features,  cols = tokens)
-//   t    = s x A^T,  u = s dY B      (rows = tokens,       cols = rank)
-//   dA^T = x^T u,    dB = dY^T t     (rows = features,     cols = rank, reduced over tokens)
-// with the fp32 intermediates t and u split into bf16 hi + lo parts so that the adapter
-// terms keep close to fp32 accuracy through bf16 tensor-core inputs.
+// with the fp32 t = s x A^T and u = s dY B (computed in lowrank.cuh) split into bf16 hi + lo
+// parts, run as extra k-blocks of the same accumulator, so that the adapter terms keep close
+// to fp32 accuracy through bf16 tensor-core inputs.
 //
-// Warp roles: warp 0 (and warps 10.. when kTmaWarps > 1) issue TMA loads, warp 1 allocates TMEM
-// and issues MMAs, warps 2-9 run the dequant producer (two groups of four warps on alternate
-// k-blocks) and then the epilogue (each group drains half of the accumulator columns).
+// Warp roles: warps 0 and 10.. (kTmaWarps of them) issue the TMA loads of alternate k-blocks,
+// warp 1 allocates TMEM and (lane 0) issues the MMAs, warps 2-9 run the dequant producer (two
+// groups of four warps on alternate k-blocks) and then the epilogue (each group drains half of
+// the accumulator columns).  Per pipeline stage s:
+//   full[s]   the B tile (and a TMA-loaded A tile) has landed;
+//   cfull[s]  the codes have landed (shared-memory A), or a plain arrive: producers may start;
+//   prod[s]   the producers wrote the A tile, after they also saw full[s];
+//   empty[s]  the MMAs that read stage s completed (tcgen05.commit).
 #pragma once
 
 #include "nf4_device.cuh"
