@@ -138,7 +138,8 @@ int nf4_dequant(const uint8_t* codes, const uint8_t* scale_codes, const float* c
  *   x       : bf16[M][K]          A : bf16[r][K]          B : bf16[N][r]
  *   y       : bf16[M][N], written
  *   t_saved : float[M][r], written: t = s x A^T (fp32), kept by the caller for the backward
- * W' is produced tile by tile in shared memory from the codes and is never written to HBM.
+ * W' is produced tile by tile on chip (in tensor memory for 256-token tiles, else in shared
+ * memory) from the codes and is never written to HBM.
  * Requirements: K % 8 == 0, N % 8 == 0, r % 8 == 0, 8 <= r <= 256, bf16 and code pointers
  * 16-byte aligned.  Accuracy: fp32 accumulation of exact bf16 products; the adapter term uses
  * t split into bf16 hi + lo parts.  Workspace: qlora_linear_fwd_workspace_bytes(M, K, N, r)
