@@ -24,7 +24,11 @@ quantize_nf4_dq        brute-force exact-rational recomputation on tiny
                        tensors; storage arithmetic of the pages; exact-zero
                        blocks; reconstruction error bound of the scales
 dequant_nf4_dq         worked lookup (reconstruction 0.3218604028); exact
-                       zeros; closed-form single-block cases
+                       zeros; closed-form single-block cases; 600 blocks of
+                       distinct scales (3 groups) against exact rationals
+bf16_rn_bits           torch's fp32 -> bf16 cast on every tie pattern (both
+                       parities of the kept bit) and neighbours; exact
+                       rational nearest-even rounding on random patterns
 =====================  ======================================================
 """
 

@@ -194,3 +194,148 @@ def test_dequant_scales_follow_fma_definition():
         exact = Fraction(float(nf4.e4m3_decode(codes[i]))) * Fraction(float(c2[i // 256])) \
             + Fraction(float(mean))
         assert s[i] == nf4.f32_from_rational(exact)
+
+
+# ----------------------------------------------------------------------------------------
+# dequant over many blocks with distinct scales, against exact rationals
+# ----------------------------------------------------------------------------------------
+
+def _e4m3_value(byte: int) -> Fraction:
+    """E4M3 (bias 7) value of a byte from the format's closed form, as an exact rational."""
+    sign = -1 if byte & 0x80 else 1
+    e, m = (byte >> 3) & 15, byte & 7
+    mag = Fraction(m, 512) if e == 0 else Fraction(8 + m, 8) * Fraction(2) ** (e - 7)
+    return sign * mag
+
+
+def _bf16_rn_rational(x: Fraction) -> int:
+    """bf16 bit pattern nearest to the exact rational x, ties to the even significand
+    (restated from the format: 1 sign, 8 exponent bits, 7 stored mantissa bits)."""
+    if x == 0:
+        return 0
+    sign = 0x8000 if x < 0 else 0
+    a = abs(x)
+    e = 0
+    while a >= 2:
+        a /= 2; e += 1
+    while a < 1:
+        a *= 2; e -= 1
+    e = max(e, -126)                       # subnormal range: spacing 2^-133
+    scaled = abs(x) / Fraction(2) ** (e - 7)   # significand in units of the last place
+    lo = scaled.numerator // scaled.denominator
+    rem = scaled - lo
+    up = rem > Fraction(1, 2) or (rem == Fraction(1, 2) and lo % 2 == 1)
+    mant = lo + (1 if up else 0)           # 128..256 for normals (256 carries into e + 1)
+    if mant >= 256:
+        mant //= 2; e += 1
+    if mant < 128:                         # subnormal
+        return sign | mant
+    return sign | ((e + 127) << 7) | (mant - 128)
+
+
+def _dequant_exact(packed, scale_codes, c2, mean, numel):
+    """W'_e = bf16(fp32(q[code_e] * fp32(e4m3(e_b) * c2_g + mean))) with b = e // 64 and
+    g = b // 256, every rounding done from exact rationals."""
+    q = [Fraction(float(v)) for v in nf4.nf4_codebook()]
+    codes = nf4.unpack_codes(packed, numel)
+    scales = {}
+    out = np.empty(numel, np.uint16)
+    for e in range(numel):
+        b = e // 64
+        if b not in scales:
+            exact = _e4m3_value(int(scale_codes[b])) * Fraction(float(c2[b // 256])) + Fraction(float(mean))
+            scales[b] = Fraction(float(nf4.f32_from_rational(exact)))
+        prod = Fraction(float(nf4.f32_from_rational(q[int(codes[e])] * scales[b])))
+        out[e] = _bf16_rn_rational(prod)
+    return out
+
+
+def _multiblock_weight(nblocks, seed):
+    """bf16 weights whose blocks have widely different absmax values, so that the 8-bit
+    scale codes of neighbouring blocks (and the constants of neighbouring groups) differ."""
+    rng = np.random.default_rng(seed)
+    std = np.exp(rng.uniform(np.log(1e-3), np.log(0.1), nblocks)).astype(np.float32)
+    w = rng.standard_normal((nblocks, 64)).astype(np.float32) * std[:, None]
+    return _bf16_exact(w.ravel())
+
+
+def test_dequant_many_blocks_matches_exact_rationals():
+    """600 blocks (3 groups of 256, the last partial) with distinct scales: every weight
+    uses its own block's scale and its group's constant.  Pins the per-element block and
+    group indexing of the dequant, which single-block or constant-scale cases cannot."""
+    w = _multiblock_weight(600, 21)
+    qd = nf4.quantize_nf4_dq(w)
+    assert len(set(qd["scale_codes"].tolist())) > 50 and qd["c2"].size == 3
+    got = nf4.dequant_nf4_dq(qd["codes"], qd["scale_codes"], qd["c2"], qd["mean"], w.size)
+    want = _dequant_exact(qd["codes"], qd["scale_codes"], qd["c2"], qd["mean"], w.size)
+    assert np.array_equal(got, want)
+
+
+def test_dequant_pin_rejects_a_planted_block_index_mistake():
+    """The exact-rational pin above fails for an oracle dequant that indexes the block
+    scale by element // 256 instead of element // 64."""
+    w = _multiblock_weight(600, 22)
+    qd = nf4.quantize_nf4_dq(w)
+    q = nf4.nf4_codebook()
+    codes = nf4.unpack_codes(qd["codes"], w.size)
+    s = nf4.block_scales(qd["scale_codes"], qd["c2"], qd["mean"])
+    planted = nf4.bf16_rn_bits((q[codes].astype(np.float64)
+                                * s[np.arange(w.size) // 256].astype(np.float64)).astype(np.float32))
+    want = _dequant_exact(qd["codes"], qd["scale_codes"], qd["c2"], qd["mean"], w.size)
+    assert not np.array_equal(planted, want)
+
+
+# ----------------------------------------------------------------------------------------
+# fp32 -> bf16 rounding: ties to even
+# ----------------------------------------------------------------------------------------
+
+def _tie_patterns():
+    """fp32 bit patterns whose dropped low half is exactly 0x8000 (a tie), with both
+    parities of the kept last bit, over every exponent and both signs; plus neighbours
+    0x7FFF / 0x8001 of each."""
+    rng = np.random.default_rng(3)
+    hi = np.concatenate([np.arange(0, 0x7F80, dtype=np.uint32),            # finite, +
+                         rng.integers(0x8000, 0xFF80, 20000).astype(np.uint32)])
+    pats = []
+    for low in (0x8000, 0x7FFF, 0x8001, 0x0000, 0xFFFF):
+        pats.append((hi << np.uint32(16)) | np.uint32(low))
+    return np.concatenate(pats)
+
+
+def test_bf16_rounding_matches_torch_cast_on_ties():
+    import torch
+    bits = _tie_patterns()
+    x = bits.view(np.float32)
+    x = x[np.isfinite(x)]
+    got = nf4.bf16_rn_bits(x)
+    want = torch.from_numpy(x.copy()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(got, want)
+    # both parities of the kept bit really occur among the ties
+    ties = (x.view(np.uint32) & np.uint32(0xFFFF)) == np.uint32(0x8000)
+    kept = (x.view(np.uint32) >> np.uint32(16)) & np.uint32(1)
+    assert np.any(ties & (kept == 0)) and np.any(ties & (kept == 1))
+
+
+def test_bf16_rounding_matches_exact_rationals():
+    rng = np.random.default_rng(8)
+    bits = np.concatenate([
+        (rng.integers(0x0080, 0x7F00, 4000).astype(np.uint32) << np.uint32(16)) | np.uint32(0x8000),
+        rng.integers(0, 0x7F000000, 4000).astype(np.uint32),
+        rng.integers(0x80000000, 0xFF000000, 2000).astype(np.uint32),
+        np.array([0x00008000, 0x00018000, 0x80008000, 0x3F808000, 0x3F818000], np.uint32),
+    ])
+    x = bits.view(np.float32)
+    got = nf4.bf16_rn_bits(x)
+    for xi, gi in zip(x, got):
+        assert int(gi) == _bf16_rn_rational(Fraction(float(xi))), hex(int(np.float32(xi).view(np.uint32)))
+
+
+def test_bf16_pin_rejects_round_half_up():
+    """The pins above fail for a rounding that drops the kept-bit term (round half up)."""
+    import torch
+    x = _tie_patterns().view(np.float32)
+    x = x[np.isfinite(x)]
+    b = x.view(np.uint32).astype(np.uint64)
+    planted = ((b + np.uint64(0x7FFF) + np.uint64(1)) >> np.uint64(16)).astype(np.uint16)
+    want = torch.from_numpy(x.copy()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert not np.array_equal(planted, want)
