@@ -16,6 +16,13 @@ roofline of the dominant kernel (timed live with CUDA events around its launches
 oracle baseline, an end-to-end run through host buffers and the SM clocks seen during the
 timed region are reported on the same JSON line.
 
+Extra rows on the same line (rank 0, one GPU): the LLaMA-7B block at 512 tokens, the
+quantize / dequant sweep over the 80-layer 65B-shaped stack (bytes per weight, GB/s), and the
+robust 4000x3000 weight over ranks r in {8, 64, 256} and token counts M in {1, 16, 512, 16384}
+(with the HBM roofline where M <= 16).
+
+--gpus N (N > 1) without a launcher re-executes itself under torch.distributed.run with N
+ranks on this node; under a launcher the world size must equal N.
 --impl reference times the CPU oracle (oracle/) on a bounded sample of the same workload.
 """
 
@@ -44,6 +51,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # Algorithmic bytes per weight: quantize reads bf16 (2 B) and writes codes (0.5 B), scale
 # codes (1/64 B) and group constants (4/(64*256) B); dequant reads the latter and writes bf16.
 CODEC_BYTES_PER_WEIGHT = 2.0 + 0.5 + 1.0 / 64 + 4.0 / (64 * 256)
+# kernels one nf4_quantize_dq call launches
+QUANTIZE_LAUNCHES = 4
 
 
 def linears():
@@ -67,6 +76,20 @@ def load_peaks():
         return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
     except Exception:
         return dict(FALLBACK_PEAKS), "fallback"
+
+
+def pick_bf16_peak(peaks: dict, clocks: dict):
+    """The bf16 tensor peak a kernel timed in this run is measured against.
+
+    MEASURED_PEAKS.json holds a burst figure (a short matmul at full clock) and a sustained
+    one (a seconds-long loop that settles under the power cap at a lower clock).  The peak
+    that applies is the one whose clock the timed region actually ran at: the burst figure
+    when the median SM clock sampled during the timed region is within 10 % of the maximum
+    (or was not sampled), else the sustained figure."""
+    sm, smax = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
+    if sm is None or not smax or sm >= 0.9 * smax:
+        return peaks["bf16_tflops"], "burst"
+    return peaks["bf16_tflops_sustained"], "sustained"
 
 
 # ------------------------------------------------------------------------------------------
@@ -297,6 +320,61 @@ def make_events(n_linears):
             for _ in range(n_linears)]
 
 
+class CudaTimer:
+    """Device time between two CUDA events on the current stream."""
+
+    def __init__(self):
+        import torch
+        self.t0 = torch.cuda.Event(enable_timing=True)
+        self.t1 = torch.cuda.Event(enable_timing=True)
+
+    def start(self):
+        self.t0.record()
+
+    def stop(self):
+        self.t1.record()
+
+    def elapsed_ms(self) -> float:
+        return self.t0.elapsed_time(self.t1)
+
+
+def timed_region(step, steps: int, warmup: int, dist, sync, timer, reduce_max, on_start=None, on_stop=None):
+    """The rank orchestration of every timed run: `warmup` untimed steps, a barrier and a
+    synchronize, `steps` timed steps (step(k) gets the step index), a synchronize and a
+    barrier, then the elapsed time reduced to its maximum over the ranks.  Every rank takes
+    the same collective calls in the same order.  `dist` is None on one rank."""
+    for _ in range(warmup):
+        step(None)
+    sync()
+    if dist is not None:
+        dist.barrier()
+    sync()
+    if on_start:
+        on_start()
+    timer.start()
+    for k in range(steps):
+        step(k)
+    timer.stop()
+    sync()
+    if on_stop:
+        on_stop()
+    if dist is not None:
+        dist.barrier()
+    return reduce_max(timer.elapsed_ms())
+
+
+def make_reduce_max(dist, device):
+    """Max over ranks of a host float, through a one-element tensor on `device`."""
+    def reduce_max(v: float) -> float:
+        if dist is None:
+            return v
+        import torch
+        t = torch.tensor([v], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+    return reduce_max
+
+
 def ours(args, rank, world, dev_index):
     import torch
     import bit_nf4_quantized_dq_b200 as q
@@ -312,44 +390,26 @@ def ours(args, rank, world, dev_index):
         import torch.distributed as dist
     from bit_nf4_quantized_dq_b200.dp import allreduce_adapter_grads
 
-    def allreduce_grads(b):
-        if dist is not None:
-            allreduce_adapter_grads([b.dA, b.dB])
-
     stream = torch.cuda.current_stream().cuda_stream
+    ev_steps = [make_events(len(bufs)) for _ in range(args.steps)]
 
-    def step(evs=None):
+    def step(k):
+        evs = ev_steps[k] if k is not None else None
         for i, b in enumerate(bufs):
             run_linear(L, b, wdq, stream, evs[i] if evs else None)
-            allreduce_grads(b)
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    q.check_device_error()
+            if dist is not None:
+                allreduce_adapter_grads([b.dA, b.dB])
 
     # ------------------------------------------------ device-timed run (inputs resident in HBM)
-    ev_steps = [make_events(len(bufs)) for _ in range(args.steps)]
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = NvmlClockSampler(dev_index)
-    if dist is not None:
-        dist.barrier()
-    torch.cuda.synchronize()
-    clocks.start()
-    t0.record()
-    for k in range(args.steps):
-        step(ev_steps[k])
-    t1.record()
-    torch.cuda.synchronize()
-    clock_info = clocks.stop()
-    if dist is not None:
-        dist.barrier()
+    clock_info = {}
+
+    def stop_clocks():
+        clock_info.update(clocks.stop())
+
+    elapsed_ms = timed_region(step, args.steps, args.warmup, dist, torch.cuda.synchronize, CudaTimer(),
+                              make_reduce_max(dist, dev), on_start=clocks.start, on_stop=stop_clocks)
     q.check_device_error()
-    elapsed_ms = t0.elapsed_time(t1)
-    if dist is not None:
-        tt = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(tt.item())
     ms_per_step = elapsed_ms / args.steps
 
     # per-stage totals over the timed steps
@@ -381,6 +441,12 @@ def ours(args, rank, world, dev_index):
     }
     rows["quantize_frac_hbm"] = rows["quantize_gbs"] / peaks["hbm_gbs"]
     rows["dequant_frac_hbm"] = rows["dequant_gbs"] / peaks["hbm_gbs"]
+    linear_ms = sum(acc[k] for k in ("fwd_down", "fwd_fused", "bwd_prep", "bwd_up", "dx_fused", "dA", "dB")) / K
+    rows["linear_fwd_bwd_tflops"] = step_flops() / (linear_ms * 1e9)
+    peak, which = pick_bf16_peak(peaks, clock_info)
+    rows["fwd_fused_frac"] = rows["fwd_fused_tflops"] / peak
+    rows["dx_fused_frac"] = rows["dx_fused_tflops"] / peak
+    rows["linear_fwd_bwd_frac"] = rows["linear_fwd_bwd_tflops"] / peak
     # dominant kernel: the fused dequant GEMM with the larger total time
     if acc["fwd_fused"] >= acc["dx_fused"]:
         dom, dom_flops, dom_ms = "fused forward GEMM (NF4 dequant producer + tcgen05)", fused_fwd_flops, acc["fwd_fused"]
@@ -388,18 +454,27 @@ def ours(args, rank, world, dev_index):
     else:
         dom, dom_flops, dom_ms = "fused dX GEMM (NF4 dequant producer + tcgen05)", fused_dx_flops, acc["dx_fused"]
         traffic = fused_traffic("dx")
-    launches_per_linear = [b.plan["fwd_launches"] + b.plan["bwd_launches"] + 4 + 1 for b in bufs]
+    launches_per_linear = [b.plan["fwd_launches"] + b.plan["bwd_launches"] + QUANTIZE_LAUNCHES + 1 for b in bufs]
     achieved = dom_flops / (dom_ms / K) / 1e9
-    roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peaks["bf16_tflops_sustained"],
-                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops_sustained"],
-                "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step)",
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak,
+                "peak_source": (f"{peak_src} bf16 {which} (median SM clock {clock_info.get('sm_mhz')} MHz of "
+                                f"{clock_info.get('sm_max_mhz')} during the timed region)"),
+                "frac_vs_burst": achieved / peaks["bf16_tflops"],
+                "frac_vs_sustained": achieved / peaks["bf16_tflops_sustained"],
                 "traffic": traffic, "traffic_unit": "bytes per launch (DRAM read + write, ncu)",
-                "launches_per_step": len(lins), "avg_launch_ms": dom_ms / K / len(lins)}
+                "launches_per_step": len(lins), "avg_launch_ms": dom_ms / K / len(lins),
+                "algorithmic_flops_per_launch": dom_flops / len(lins)}
 
     # ------------------------------------------------ end to end through host buffers
     e2e = None
     if not args.no_e2e:
-        e2e = end_to_end(args, bufs, wdq, L, stream, dist, dev)
+        e2e = end_to_end(args, bufs, wdq, L, dist, dev)
+
+    extra = {}
+    if world == 1 and not args.no_extra:
+        del ev_steps
+        extra = extra_rows(args, L, dev, peaks, peak)
 
     flops_all = step_flops() * world
     value = flops_all / (ms_per_step / 1e3) / 1e12
@@ -413,13 +488,19 @@ def ours(args, rank, world, dev_index):
                    "step": "per linear: quantize W, dequant W, fused fwd, bwd (dX, dA, dB)"},
         "rows": rows, "roofline": roofline, "gpu_launches": sum(launches_per_linear) * K, "clocks": clock_info,
     }
+    if extra:
+        out["rows"].update(extra)
     if e2e is not None:
         out["e2e"] = e2e
     return out
 
 
-def end_to_end(args, bufs, wdq, L, stream, dist, dev):
-    """Same step through the C ABI with pinned host inputs / outputs copied every step."""
+def end_to_end(args, bufs, wdq, L, dist, dev):
+    """The same step through the C ABI with the inputs copied in from pinned host buffers and
+    the outputs copied back every step.  Host-to-device copies run on one stream, the
+    compute on the current stream and device-to-host copies on a third, ordered per linear
+    by events, so that linear i+1's inputs and linear i-1's outputs move while linear i
+    computes."""
     import torch
     from bit_nf4_quantized_dq_b200.dp import allreduce_adapter_grads
     host_in, host_out = [], []
@@ -432,37 +513,187 @@ def end_to_end(args, bufs, wdq, L, stream, dist, dev):
         host_out.append(ho)
         h2d += sum(v.numel() * v.element_size() for v in hi.values())
         d2h += sum(v.numel() * v.element_size() for v in ho.values())
+    compute = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    n = len(bufs)
+    ev_in = [torch.cuda.Event() for _ in range(n)]
+    ev_done = [torch.cuda.Event() for _ in range(n)]
+    ev_out = [torch.cuda.Event() for _ in range(n)]
 
-    def step():
-        for b, hi, ho in zip(bufs, host_in, host_out):
-            for k, v in hi.items():
-                getattr(b, k).copy_(v, non_blocking=True)
-            run_linear(L, b, wdq, stream)
+    def step(_k):
+        for i, (b, hi, ho) in enumerate(zip(bufs, host_in, host_out)):
+            s_in.wait_event(ev_done[i])          # the previous step's linear i no longer reads them
+            with torch.cuda.stream(s_in):
+                for k, v in hi.items():
+                    getattr(b, k).copy_(v, non_blocking=True)
+            ev_in[i].record(s_in)
+            compute.wait_event(ev_in[i])
+            compute.wait_event(ev_out[i])        # the previous step's outputs of linear i are copied out
+            run_linear(L, b, wdq, compute.cuda_stream)
             if dist is not None:
                 allreduce_adapter_grads([b.dA, b.dB])
-            for k, v in ho.items():
-                v.copy_(getattr(b, k), non_blocking=True)
+            ev_done[i].record(compute)
+            s_out.wait_event(ev_done[i])
+            with torch.cuda.stream(s_out):
+                for k, v in ho.items():
+                    v.copy_(getattr(b, k), non_blocking=True)
+            ev_out[i].record(s_out)
+        for i in range(n):
+            compute.wait_event(ev_out[i])        # the step ends when its last output is on the host
 
-    step()
-    torch.cuda.synchronize()
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if dist is not None:
-        dist.barrier()
-    torch.cuda.synchronize()
-    t0.record()
-    for _ in range(args.steps):
-        step()
-    t1.record()
-    torch.cuda.synchronize()
-    ms = t0.elapsed_time(t1)
-    if dist is not None:
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = timed_region(step, args.steps, 1, dist, torch.cuda.synchronize, CudaTimer(), make_reduce_max(dist, dev))
     world = dist.get_world_size() if dist is not None else 1
     value = step_flops() * world / (ms / args.steps / 1e3) / 1e12
     return {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "ms_per_step": ms / args.steps}
+            "ms_per_step": ms / args.steps,
+            "copies": "pinned host buffers; H2D, compute and D2H on three streams, overlapped across linears"}
+
+
+# ------------------------------------------------------------------------------------------
+# extra rows: the 512-token LLaMA-7B block, the 65B stack codec sweep, the robust weight
+# ------------------------------------------------------------------------------------------
+def _time_calls(fn, reps: int, warmup: int = 2) -> float:
+    """Mean device time in ms of fn() over `reps` calls on the current stream."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    t = CudaTimer()
+    torch.cuda.synchronize()
+    t.start()
+    for _ in range(reps):
+        fn()
+    t.stop()
+    torch.cuda.synchronize()
+    return t.elapsed_ms() / reps
+
+
+def rows_llama7b_512(L, dev, peak):
+    """The seven linears of a LLaMA-7B block at 512 tokens (r = 64): the same step as the
+    headline (quantize, dequant, fwd, bwd per linear)."""
+    import torch
+    import synth
+    lins = synth.LLAMA7B
+    M = 512
+    bufs = [LinearBufs(l, M, R, 2000 + i, dev) for i, l in enumerate(lins)]
+    wdq = torch.empty(max(l.N * l.K for l in lins), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream().cuda_stream
+
+    def step():
+        for b in bufs:
+            run_linear(L, b, wdq, stream)
+
+    ms = _time_calls(step, 10, 3)
+    flops = sum(linear_flops(M, l.N, l.K, R) for l in lins)
+    return {"workload": "llama7b_block_512tok", "ms_per_step": ms, "tflops": flops / (ms * 1e9),
+            "frac": flops / (ms * 1e9) / peak,
+            "note": "step = quantize + dequant + fwd + bwd of the 7 linears; flops = 4MNK + 6MKr + 6MNr"}
+
+
+def rows_stack65b(L, dev, hbm_gbs, layers: int):
+    """Quantize and dequant, layer by layer, of `layers` layers of the 65B-shaped stack (each
+    layer: 4 x 8192x8192, 3 x 22016x8192, W ~ N(0, 0.015^2) drawn per layer on the GPU)."""
+    import torch
+    import synth
+    import bit_nf4_quantized_dq_b200 as q
+    shapes = synth.STACK65B_LAYER
+    big = max(l.N * l.K for l in shapes)
+    W = torch.empty(big, dtype=torch.bfloat16, device=dev)
+    out = torch.empty(big, dtype=torch.bfloat16, device=dev)
+    nb_big = (big + 63) // 64
+    codes = torch.empty(32 * nb_big, dtype=torch.uint8, device=dev)
+    sc = torch.empty(nb_big, dtype=torch.uint8, device=dev)
+    c2 = torch.empty((nb_big + 255) // 256, dtype=torch.float32, device=dev)
+    mean = torch.empty(1, dtype=torch.float32, device=dev)
+    ws = torch.empty(L.nf4_quantize_workspace_bytes(big), dtype=torch.uint8, device=dev)
+    st = _stream_arg()
+    g = torch.Generator(device=dev)
+    tq = td = 0.0
+    nweights = nbytes = 0
+    for layer in range(layers):
+        for j, l in enumerate(shapes):
+            numel = l.N * l.K
+            g.manual_seed(synth.seed_for(4, layer * 7 + j))
+            Wv = W[:numel]
+            Wv.copy_(torch.randn(numel, generator=g, device=dev) * 0.015)
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            e[0].record()
+            rc = L.nf4_quantize_dq(_p(Wv), numel, _p(codes), _p(sc), _p(c2), _p(mean), _p(ws), ws.numel(), st)
+            e[1].record()
+            rc |= L.nf4_dequant(_p(codes), _p(sc), _p(c2), _p(mean), numel, _p(out), st)
+            e[2].record()
+            if rc != 0:
+                raise RuntimeError(L.qnf4_last_error().decode())
+            torch.cuda.synchronize()
+            tq += e[0].elapsed_time(e[1])
+            td += e[1].elapsed_time(e[2])
+            nb = (numel + 63) // 64
+            nweights += numel
+            nbytes += 32 * nb + nb + 4 * ((nb + 255) // 256) + 4
+    q.check_device_error()
+    gb = nweights * CODEC_BYTES_PER_WEIGHT / 1e9
+    return {"workload": "stack65b_codec", "layers_timed": layers, "layers_in_stack": 80, "weights": nweights,
+            "stored_bits_per_weight": nbytes * 8 / nweights,
+            "stored_bits_per_weight_expected": 4.126953125, "stack_stored_gb_80_layers": nbytes * 80 / layers / 1e9,
+            "quantize_gbs": gb / (tq / 1e3), "dequant_gbs": gb / (td / 1e3),
+            "quantize_frac_hbm": gb / (tq / 1e3) / hbm_gbs, "dequant_frac_hbm": gb / (td / 1e3) / hbm_gbs,
+            "note": "algorithmic bytes 2.51587 per weight for each of quantize and dequant"}
+
+
+def _stream_arg():
+    import ctypes
+    import torch
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def linear_hbm_bytes(M, N, K, r):
+    """Algorithmic HBM bytes of one fwd + bwd: activations, codes + scales, adapters, outputs."""
+    codec = N * K * (0.5 + 1.0 / 64 + 4.0 / (64 * 256))
+    fwd = 2 * M * K + codec + 2 * r * K + 2 * N * r + 2 * M * N + 4 * M * r
+    bwd = 2 * M * N + codec + 2 * M * K + 2 * M * K + 2 * (2 * r * K + 2 * N * r) + 4 * M * r
+    return fwd + bwd
+
+
+def rows_robust(L, dev, peaks, peak):
+    """fwd + bwd on the robust 4000x3000 weight (Student-t, outlier columns, exact zeros) for
+    r in {8, 64, 256} and M in {1, 16, 512, 16384}; M <= 16 is reported against HBM."""
+    import torch
+    import synth
+    import bit_nf4_quantized_dq_b200 as q
+    N, K = 4000, 3000
+    W = synth.robust_weight_bf16(N, K, synth.seed_for(5, 0)).to(dev)
+    Q = q.nf4_quantize_dq(W)
+    out = []
+    for r in (8, 64, 256):
+        for M in (1, 16, 512, 16384):
+            inp = synth.linear_inputs(M, N, K, r, synth.seed_for(5, 10 + r + M), device=str(dev))
+            s = ALPHA / r
+            wsf = torch.empty(max(256, L.qlora_linear_fwd_workspace_bytes(M, K, N, r)), dtype=torch.uint8, device=dev)
+            wsb = torch.empty(max(256, L.qlora_linear_bwd_workspace_bytes(M, K, N, r)), dtype=torch.uint8, device=dev)
+            x, A, B, dY = inp["x"], inp["A"], inp["B"], inp["dY"]
+
+            def fb():
+                y, t = q.qlora_linear_fwd(x, Q, A, B, s, workspace=wsf)
+                q.qlora_linear_bwd(dY, x, t, Q, A, B, s, workspace=wsb)
+
+            ms = _time_calls(fb, 20 if M <= 512 else 5)
+            flops = linear_flops(M, N, K, r)
+            row = {"r": r, "M": M, "ms": ms, "tflops": flops / (ms * 1e9), "frac_tensor": flops / (ms * 1e9) / peak}
+            hb = linear_hbm_bytes(M, N, K, r)
+            row["gbs"] = hb / (ms * 1e6)
+            if M <= 16:
+                row["frac_hbm"] = row["gbs"] / peaks["hbm_gbs"]
+            out.append(row)
+    q.check_device_error()
+    return {"workload": "robust_4000x3000", "points": out,
+            "note": "fwd + bwd through the Python binding (allocating outputs); M <= 16 is HBM-bound"}
+
+
+def extra_rows(args, L, dev, peaks, peak):
+    import torch
+    torch.cuda.empty_cache()
+    return {"llama7b_512": rows_llama7b_512(L, dev, peak),
+            "stack65b": rows_stack65b(L, dev, peaks["hbm_gbs"], args.stack_layers),
+            "robust": rows_robust(L, dev, peaks, peak)}
 
 
 # ------------------------------------------------------------------------------------------
@@ -590,7 +821,27 @@ def single_case(args):
     print(json.dumps({"case": args.case, "linear": args.linear, "tokens": M_TOKENS, "ms_per_call": ms}), flush=True)
 
 
-def main():
+def launcher_command(args, argv):
+    """torch.distributed.run command that starts `args.gpus` ranks of this script on this node."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={args.gpus}",
+            "--master-addr", "127.0.0.1", f"--master-port={port}", os.path.abspath(__file__), *argv]
+
+
+def check_world(args, env) -> tuple:
+    """(rank, world, local rank) from the launcher's environment; the world size must match
+    --gpus (a silent one-rank run of `--gpus 8` would report the wrong n_gpus)."""
+    world = int(env.get("WORLD_SIZE", "1"))
+    if world != args.gpus:
+        raise SystemExit(f"bench.py: --gpus {args.gpus} but the launcher started {world} rank(s)")
+    return int(env.get("RANK", "0")), world, int(env.get("LOCAL_RANK", "0"))
+
+
+def main(argv=None):
+    argv = sys.argv[1:] if argv is None else argv
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=5)
@@ -598,25 +849,29 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end run")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the oracle sample")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the extra rows (512-token block, 65B stack sweep, robust weight)")
+    ap.add_argument("--stack-layers", type=int, default=80, help="layers of the 65B stack in the codec sweep")
     ap.add_argument("--case", choices=CASES, default=None,
                     help="run one call family on one linear only (profiling aid; prints its own line)")
     ap.add_argument("--linear", default="q", help="linear of the block used by --case")
-    args = ap.parse_args()
+    args = ap.parse_args(argv)
     if args.case:
         single_case(args)
-        return
+        return 0
+    if args.gpus < 1:
+        raise SystemExit("--gpus must be >= 1")
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        return subprocess.call(launcher_command(args, argv))
+    rank, world, local = check_world(args, os.environ)
     if args.warmup < 3 and args.impl == "ours":
         print("note: fewer than 3 warm-up steps", file=sys.stderr)
-
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
 
     if args.impl == "reference":
         out = reference(args, rank, world)
         if out is not None:
             print(json.dumps(out), flush=True)
-        return
+        return 0
 
     import torch
     if world > 1:
@@ -636,7 +891,8 @@ def main():
         if world > 1:
             import torch.distributed as dist
             dist.destroy_process_group()
+    return 0
 
 
 if __name__ == "__main__":
-    main()
+    sys.exit(main())

@@ -157,22 +157,38 @@ def nf4_quantize_dq(W: torch.Tensor, workspace: Optional[torch.Tensor] = None) -
     return NF4Tensor(codes, scale_codes, c2, mean, W.shape)
 
 
+def _check_out_buffer(t: torch.Tensor, dtype, count: int, device, name: str) -> None:
+    if not isinstance(t, torch.Tensor) or t.dtype != dtype or not t.is_contiguous() or t.device != device:
+        raise QNF4Error(f"out.{name} must be a contiguous {dtype} tensor on {device}")
+    if t.numel() < count:
+        raise QNF4Error(f"out.{name} holds {t.numel()} elements, the weight needs {count}")
+
+
 def nf4_quantize_dq_noalloc(W: torch.Tensor, out: Optional[NF4Tensor] = None) -> NF4Tensor:
     """nf4_quantize_dq without a workspace: the library's static scratch holds the absmax and
     group sums (numel <= NOALLOC_MAX_NUMEL; overlapping calls on one device race on it).  Pass
-    `out` to write into existing buffers, so that the call itself allocates nothing."""
+    `out` to write into existing buffers, so that the call itself allocates nothing; they are
+    checked against W (device, dtype, contiguity, size) before the call."""
     W = _bf16_bits(W)
     _require_cuda(W)
     numel = W.numel()
+    nb = (numel + 63) // 64
+    ng = (nb + 255) // 256
+    dev = W.device
     if out is None:
-        nb = (numel + 63) // 64
-        dev = W.device
         out = NF4Tensor(torch.empty(32 * nb, dtype=torch.uint8, device=dev),
                         torch.empty(nb, dtype=torch.uint8, device=dev),
-                        torch.empty((nb + 255) // 256, dtype=torch.float32, device=dev),
+                        torch.empty(ng, dtype=torch.float32, device=dev),
                         torch.empty(1, dtype=torch.float32, device=dev), W.shape)
-    _check(lib().nf4_quantize_dq_noalloc(_ptr(W), numel, _ptr(out.codes), _ptr(out.scale_codes), _ptr(out.c2),
-                                         _ptr(out.mean), _stream()), "nf4_quantize_dq_noalloc")
+    else:
+        _check_out_buffer(out.codes, torch.uint8, 32 * nb, dev, "codes")
+        _check_out_buffer(out.scale_codes, torch.uint8, nb, dev, "scale_codes")
+        _check_out_buffer(out.c2, torch.float32, ng, dev, "c2")
+        _check_out_buffer(out.mean, torch.float32, 1, dev, "mean")
+    with torch.cuda.device(dev):
+        _check(lib().nf4_quantize_dq_noalloc(_ptr(W), numel, _ptr(out.codes), _ptr(out.scale_codes), _ptr(out.c2),
+                                             _ptr(out.mean), _stream()), "nf4_quantize_dq_noalloc")
+    out.shape = tuple(W.shape)
     return out
 
 

@@ -3,6 +3,7 @@
 // descriptors of the 128-byte swizzled canonical layouts.
 #pragma once
 
+#include <atomic>
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -31,6 +32,21 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
   return t;
+}
+
+// Dynamic shared memory above 48 KB has to be enabled for a kernel on every device it runs on
+// (cudaFuncSetAttribute acts through the current device).  `done` holds one bit per device
+// ordinal, so each kernel sets it once per device.
+template <class Kernel>
+inline cudaError_t enable_smem_once(Kernel* kernel, int bytes, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

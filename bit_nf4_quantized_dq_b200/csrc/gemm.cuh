@@ -538,13 +538,9 @@ __global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_co
 template <int BN, bool GENERIC, bool A_TMEM = false>
 static cudaError_t launch_bn(const GemmParams& p, cudaStream_t st) {
   using C = Cfg<BN, A_TMEM>;
-  static bool configured = false;   // per process; the attribute is per function, not per device
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(qlora_gemm_kernel<BN, GENERIC, A_TMEM>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  static std::atomic<uint64_t> configured{0};
+  cudaError_t e = enable_smem_once(qlora_gemm_kernel<BN, GENERIC, A_TMEM>, C::kSmemBytes, configured);
+  if (e != cudaSuccess) return e;
   dim3 grid((p.rows + kBM - 1) / kBM, (p.cols + BN - 1) / BN, p.splits);
   qlora_gemm_kernel<BN, GENERIC, A_TMEM><<<grid, kThreads, C::kSmemBytes, st>>>(p);
   return cudaGetLastError();

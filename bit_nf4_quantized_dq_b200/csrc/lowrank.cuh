@@ -268,13 +268,9 @@ __global__ void __launch_bounds__(kLrThreads, 1) lowrank_kernel(const __grid_con
 template <int BJ, int TERMS>
 static cudaError_t launch_lowrank_t(const LowRankParams& p, cudaStream_t st) {
   using C = LrCfg<BJ, TERMS>;
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(lowrank_kernel<BJ, TERMS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  static std::atomic<uint64_t> configured{0};
+  cudaError_t e = enable_smem_once(lowrank_kernel<BJ, TERMS>, C::kSmemBytes, configured);
+  if (e != cudaSuccess) return e;
   dim3 grid((p.rows + 127) / 128, (p.cols + BJ - 1) / BJ, p.splits);
   lowrank_kernel<BJ, TERMS><<<grid, kLrThreads, C::kSmemBytes, st>>>(p);
   return cudaGetLastError();

@@ -10,7 +10,6 @@
 #include "qlora_nf4.h"
 #include "codec.cuh"
 #include "gemm.cuh"
-#include "gemm2sm.cuh"
 #include "lowrank.cuh"
 
 namespace {
@@ -273,17 +272,12 @@ int run_lowrank(const void* a_base, bool a_mn, int64_t a_inner, int64_t a_outer,
   return QNF4_OK;
 }
 
-// The fused GEMMs run on one CTA per tile; kPairTiles switches 256-token tiles to CTA pairs
-// (cta_group::2, gemm2sm.cuh).  Rows of each B-operand TMA box: a CTA of a pair loads half of
-// the 256-token tile.
-constexpr bool kPairTiles = false;
 // The fused forward keeps its A operand in tensor memory (gemm.cuh, A_TMEM) on 256-token tiles.
 constexpr bool kATmemForward = true;
-int b_box_rows(int bn) { return (kPairTiles && bn == 256) ? 128 : bn; }
+// Rows of each B-operand TMA box: one box fills one token tile.
+int b_box_rows(int bn) { return bn; }
 
-cudaError_t launch_fused(const qnf4::GemmParams& gp, int bn, cudaStream_t st) {
-  return (kPairTiles && bn == 256) ? qnf4::launch_gemm2(gp, st) : qnf4::launch_gemm(gp, bn, st);
-}
+cudaError_t launch_fused(const qnf4::GemmParams& gp, int bn, cudaStream_t st) { return qnf4::launch_gemm(gp, bn, st); }
 
 int nf4_operand(qnf4::GemmParams& gp, const uint8_t* codes, const uint8_t* scale_codes, const float* c2,
                 const float* mean, int64_t N, int64_t K) {
@@ -321,9 +315,30 @@ static __device__ __align__(256) unsigned char g_quant_scratch[kNoAllocScratchBy
 namespace {
 constexpr int kNoAllocMaxDevices = 64;
 std::mutex g_noalloc_mutex;
-void* g_noalloc_scratch[kNoAllocMaxDevices];   // device address of g_quant_scratch, per device
+struct NoAllocSlot {
+  CUcontext ctx;   // context the address was looked up in
+  void* ptr;       // device address of g_quant_scratch in that context
+};
+NoAllocSlot g_noalloc_scratch[kNoAllocMaxDevices];
 
-// One-time set-up per device: with that device current, look up the scratch's address.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+CUcontext current_context() {
+  static CtxGetCurrentFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  }
+  CUcontext c = nullptr;
+  if (fn && fn(&c) != CUDA_SUCCESS) c = nullptr;
+  return c;
+}
+
+// Set-up per device: with that device current, look up the scratch's device address.  The
+// address belongs to the device's current context, so it is looked up again whenever that
+// context differs from the one it was found in (after a cudaDeviceReset, for instance).
 int noalloc_scratch(void** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
@@ -332,13 +347,16 @@ int noalloc_scratch(void** out) {
     return fail(QNF4_ERR_UNSUPPORTED, "device ordinal %d: the static scratch supports devices 0..%d", dev,
                 kNoAllocMaxDevices - 1);
   std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (!g_noalloc_scratch[dev]) {
+  NoAllocSlot& slot = g_noalloc_scratch[dev];
+  const CUcontext ctx = current_context();
+  if (!slot.ptr || !ctx || slot.ctx != ctx) {
     void* ptr = nullptr;
     e = cudaGetSymbolAddress(&ptr, g_quant_scratch);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the quantization scratch");
-    g_noalloc_scratch[dev] = ptr;
+    slot.ptr = ptr;
+    slot.ctx = current_context();   // the lookup has made the device's context current
   }
-  *out = g_noalloc_scratch[dev];
+  *out = slot.ptr;
   return QNF4_OK;
 }
 }  // namespace
@@ -494,7 +512,7 @@ int qlora_linear_fwd(const uint16_t* x, int64_t M, int64_t K, int64_t N, const u
     gp.seg[0] = qnf4::GemmSeg{kblocks(K), k16_last(K), qnf4::kANf4K, 0, 1, 0, 0, 0};
     gp.seg[1] = qnf4::GemmSeg{kblocks(r), k16_last(r), qnf4::kATmaK, 2, 3, 0, 0, 0};
     gp.seg[2] = qnf4::GemmSeg{kblocks(r), k16_last(r), qnf4::kATmaK, 2, 4, 0, 0, 0};
-    if (kATmemForward && plan.bn == 256 && !kPairTiles) {
+    if (kATmemForward && plan.bn == 256) {
       // 256-token tiles keep the dequantized W tile (and the adapter matrix rows) in tensor
       // memory, which leaves shared memory for 6 stages instead of 4
       gp.a_tmem = 1;

@@ -106,8 +106,9 @@ int nf4_quantize_dq(const uint16_t* W, int64_t numel, uint8_t* codes, uint8_t* s
  *  - numel above QNF4_NOALLOC_MAX_NUMEL returns QNF4_ERR_UNSUPPORTED before any device work;
  *    quantize larger weights with nf4_quantize_dq and a workspace.
  *  - The first call on each device does a one-time set-up: with that device current it looks
- *    up the device address of the scratch array.  Make that first call before any stream
- *    capture begins.
+ *    up the device address of the scratch array (and looks it up again if the device's
+ *    context has been re-created since, e.g. after cudaDeviceReset).  Make that first call
+ *    before any stream capture begins.
  *  - Nothing has to start at zero: every scratch element a call reads, the same call writes
  *    first.
  *  - There is one scratch array per device, shared by every call on that device.  Calls that

@@ -102,3 +102,58 @@ def test_above_the_static_limit_is_rejected_before_device_work():
     assert L.nf4_quantize_dq_noalloc(p, MAX_NUMEL + 1, p, p, p, p, _stream()) == -2
     assert b"static scratch limit" in L.qnf4_last_error()
     assert binding.NOALLOC_MAX_NUMEL == MAX_NUMEL
+
+
+def _oracle_sampled(W_cpu, blocks):
+    """Oracle scale codes / c2 / mean of the whole weight, and the codes of `blocks` only
+    (a block's codes depend on its own 64 weights and absmax alone)."""
+    import numpy as np
+    from oracle import nf4 as onf4
+    w = W_cpu.float().numpy().ravel()
+    absmax = onf4.block_absmax(w)
+    dq = onf4.double_quantize(absmax)
+    nb = absmax.size
+    wp = np.zeros(nb * 64, np.float32)
+    wp[:w.size] = w
+    _, packed = onf4.level1_codes(wp.reshape(nb, 64)[blocks].ravel())
+    return dq, packed.reshape(len(blocks), 32)
+
+
+@pytest.mark.parametrize("numel", [MAX_NUMEL, MAX_NUMEL - 32])
+def test_size_limit_fills_the_static_scratch(numel):
+    """numel at the limit (every absmax slot and group sum of the static array in use) and
+    just below it (a ragged last block): equal to the workspace entry point bit for bit, and
+    to the oracle on the DQ parts and on sampled blocks' codes."""
+    import numpy as np
+    L = binding.lib()
+    W_cpu = synth.normal_bf16((numel,), 0.02, 7400 + (numel & 63))
+    W = W_cpu.to("cuda")
+    ref = _reference(L, W)
+    got = _noalloc(L, W, 0x99)
+    _assert_same(ref, got)
+    nb = (numel + 63) // 64
+    rng = np.random.default_rng(numel)
+    blocks = np.unique(np.concatenate([rng.choice(nb, 3000, replace=False), [0, nb - 2, nb - 1]]))
+    dq, packed = _oracle_sampled(W_cpu, blocks)
+    codes = got[0].view(-1, 32)[torch.as_tensor(blocks, device="cuda")].cpu().numpy()
+    assert np.array_equal(codes, packed)
+    assert np.array_equal(got[1].cpu().numpy(), dq["scale_codes"])
+    assert np.array_equal(got[2].cpu().numpy(), dq["c2"])
+    assert got[3].cpu().numpy()[0] == dq["mean"]
+    del W, ref, got
+    torch.cuda.empty_cache()
+
+
+def test_binding_rejects_out_buffers_too_small_for_the_weight():
+    small = binding.nf4_quantize_dq(_weight(64, 64, 7500))
+    W = _weight(640, 960, 7501)
+    with pytest.raises(binding.QNF4Error, match="codes"):
+        binding.nf4_quantize_dq_noalloc(W, out=small)
+    wrong = binding.nf4_quantize_dq(W)
+    wrong.c2 = wrong.c2.to(torch.float64)
+    with pytest.raises(binding.QNF4Error, match="c2"):
+        binding.nf4_quantize_dq_noalloc(W, out=wrong)
+    # a correctly sized buffer from a weight of another shape is accepted and takes W's shape
+    other = binding.nf4_quantize_dq(_weight(960, 640, 7502))
+    got = binding.nf4_quantize_dq_noalloc(W, out=other)
+    assert got.shape == (640, 960)
