@@ -147,3 +147,75 @@ def test_e4m3_encoders_match_oracle():
 def test_zero_size_is_rejected():
     with pytest.raises(q.QNF4Error):
         q.nf4_quantize_dq(torch.zeros(0, dtype=torch.bfloat16, device="cuda"))
+
+
+def _reachable_blocks(c_exponents=(0, -20, 30)):
+    """Blocks [c or -c, w1..w63] covering, for every bf16 absmax significand c (128 of them, at
+    each exponent in `c_exponents`), every bf16 weight w with |w| <= c whose exponent lies
+    within 10 binades of c's (both signs), plus exact zeros.  The normalised value
+    n = fp32(w / c) depends only on the two significands and the exponent gap, and any gap
+    above 5 puts |n| below 1/32, far under the smallest midpoint (code 7), so these blocks
+    reach every normalised value that can decide a code."""
+    blocks = []
+    mant = np.arange(128, dtype=np.float64)
+    for ec in c_exponents:
+        for mc in range(128):
+            c = (1.0 + mc / 128.0) * 2.0 ** ec
+            ws = []
+            for k in range(11):
+                w = (1.0 + mant / 128.0) * 2.0 ** (ec - k)
+                w = w[w <= c]
+                ws += [w, -w]
+            ws.append(np.zeros(5))
+            w = np.concatenate(ws).astype(np.float32)
+            w = np.pad(w, (0, (-w.size) % 63))
+            lead = np.full((w.size // 63, 1), c if mc % 2 == 0 else -c, np.float32)
+            blocks.append(np.concatenate([lead, w.reshape(-1, 63)], axis=1))
+    return np.concatenate(blocks).ravel()
+
+
+def test_nearest_level_exhaustive_over_reachable_quotients():
+    """Every normalised value a bf16 weight and a bf16 absmax can produce (and that can decide
+    a code) goes through the GPU quantizer: codes, scale codes, c2 and mean bit-exact."""
+    data = _reachable_blocks()
+    assert data.size > 1_000_000
+    ref, _ = _assert_codec_equal(torch.from_numpy(data).to(torch.bfloat16))
+    codes = onf4.unpack_codes(ref["codes"], data.size)
+    assert set(np.unique(codes).tolist()) == set(range(16))
+
+
+def test_e4m3_hardware_and_software_encoders_agree_on_every_fp32_in_unit_interval():
+    """All 2 x (0x3F800000 + 1) fp32 values in [-1, 1], in chunks, through both encoders on the
+    GPU (the hardware conversion is the one the quantizer uses)."""
+    step = 1 << 27
+    for sign in (0, 0x80000000):
+        lo, hi = 0, 0x3F800000 + 1
+        for a in range(lo, hi, step):
+            b = min(hi, a + step)
+            bits = torch.arange(a, b, dtype=torch.int64, device="cuda") | sign
+            v = bits.to(torch.int32).view(torch.float32) if sign == 0 else \
+                (bits - (1 << 32)).to(torch.int32).view(torch.float32)
+            hw = q.e4m3_encode(v, 0)
+            sw = q.e4m3_encode(v, 1)
+            bad = int((hw != sw).sum())
+            assert bad == 0, f"{bad} mismatches in [{a:#x}, {b:#x}) sign {sign:#x}"
+    torch.cuda.synchronize()
+
+
+def test_e4m3_encoders_match_oracle_near_every_midpoint():
+    """Every fp32 within 64 ulp of each midpoint between neighbouring E4M3 values in [0, 1]
+    (and their negatives), plus every E4M3 value's own neighbourhood."""
+    pos = onf4.e4m3_decode(np.arange(127))
+    pos = pos[pos <= 1.0]
+    pts = np.concatenate([(pos[:-1] + pos[1:]) / 2, pos]).astype(np.float32)
+    bits = pts.view(np.uint32).astype(np.int64)
+    offs = np.arange(-64, 65, dtype=np.int64)
+    allb = (bits[:, None] + offs[None, :]).ravel()
+    allb = allb[(allb >= 0) & (allb <= 0x3F800000)]
+    v = allb.astype(np.uint32).view(np.float32)
+    v = np.concatenate([v, -v])
+    want = onf4.e4m3_encode_rn(v)
+    vt = torch.from_numpy(v).cuda()
+    for mode in (0, 1):
+        got = q.e4m3_encode(vt, mode).cpu().numpy()
+        assert np.array_equal(got, want), f"mode {mode}: {int((got != want).sum())} mismatches"

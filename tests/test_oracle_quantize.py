@@ -339,3 +339,23 @@ def test_bf16_pin_rejects_round_half_up():
     planted = ((b + np.uint64(0x7FFF) + np.uint64(1)) >> np.uint64(16)).astype(np.uint16)
     want = torch.from_numpy(x.copy()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
     assert not np.array_equal(planted, want)
+
+
+def test_normalised_value_is_the_correctly_rounded_quotient():
+    """The oracle forms n = fp32(w / c) through a float64 quotient; for every pair of bf16
+    significands (and exponent gaps 0, 1, 5) it equals the exact quotient rounded once to
+    fp32 (ties to even), computed from rationals."""
+    mant = [1 + Fraction(m, 128) for m in range(128)]
+    ws, cs, exact = [], [], []
+    for gap in (0, 1, 5):
+        for mw in mant:
+            for mc in mant:
+                w = mw * Fraction(1, 2 ** gap)
+                if w > mc:
+                    continue
+                ws.append(float(w)); cs.append(float(mc)); exact.append(w / mc)
+    w = np.array(ws, np.float32); c = np.array(cs, np.float32)
+    n = (w.astype(np.float64) / c.astype(np.float64)).astype(np.float32)
+    rng = np.random.default_rng(0)
+    for i in rng.choice(len(exact), 6000, replace=False):
+        assert n[i] == nf4.f32_from_rational(exact[i])
