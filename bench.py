@@ -52,7 +52,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # codes (1/64 B) and group constants (4/(64*256) B); dequant reads the latter and writes bf16.
 CODEC_BYTES_PER_WEIGHT = 2.0 + 0.5 + 1.0 / 64 + 4.0 / (64 * 256)
 # kernels one nf4_quantize_dq call launches
-QUANTIZE_LAUNCHES = 4
+QUANTIZE_LAUNCHES = 2
 
 
 def linears():

@@ -55,108 +55,224 @@ __device__ __forceinline__ uint32_t nearest_code(float n, const BucketEntry (*ta
   return e.base + (n > e.thr ? 1u : 0u);
 }
 
-// Correctly rounded quotient w / c from y = RN(1/c): q0 = RN(w y), the remainder w - c q0 is
-// exact by one fused multiply-add, and RN(q0 + remainder * y) is RN(w / c).  This is
-// Markstein's correction step (P. Markstein, "Computation of elementary functions on the IBM
-// RISC System/6000 processor", IBM J. Res. Develop. 34(1), 1990; the theorem on Markstein's
-// iteration in Muller et al., "Handbook of Floating-Point Arithmetic"): with y within half an
-// ulp of 1/c and q0 within one ulp of w/c, the corrected quotient is the correctly rounded one,
-// as long as no intermediate leaves the normal range.  Callers keep 2^-100 <= c <= 2^100 and
-// |w| <= c, which guarantees that (a tiny quotient may be subnormal, and such an n is far
-// below every midpoint, so its code does not depend on the last bits).
-__device__ __forceinline__ float div_rn_by_recip(float w, float c, float y) {
-  const float q0 = __fmul_rn(w, y);
-  const float r = __fmaf_rn(-c, q0, w);
-  return __fmaf_rn(r, y, q0);
+// Correctly rounded n = fp32(w / c) for bf16 w and c without a division per weight.
+//
+// w / c = (mw / mc) 2^k with 8-bit integer significands mw, mc.  Such a quotient is never an
+// fp32 rounding midpoint, and is at least 2^-32 (relative) away from every one: the gap to
+// a midpoint (2M + 1) 2^(E - 24) is 2^(E - 24) |mw 2^j - mc (2M + 1)| / mc, a nonzero integer
+// over mc <= 255.  So any approximation of w / c within 2^-40 (relative) rounds to the same
+// fp32 value.  With the reciprocal as an unevaluated sum y_hi + y_lo (y_hi = RN(1/c), the
+// remainder 1 - c y_hi exact by a fused multiply-add, y_lo = RN(remainder * y_hi)), y_hi + y_lo
+// is within about 2^-46 of 1/c, and fma(w, y_hi, RN(w y_lo)) rounds a value within about
+// 2^-45 of w / c, once: the result is RN(w / c).  Valid while c, 1/c and y_lo stay normal;
+// callers keep 2^-100 <= c <= 2^100 and |w| <= c (a subnormal n can only be a tiny one, far
+// below every midpoint between levels, whose code cannot change).
+struct Recip2 {
+  float hi, lo;
+};
+__device__ __forceinline__ Recip2 recip2(float c) {
+  const float hi = __frcp_rn(c);
+  const float rem = __fmaf_rn(-c, hi, 1.0f);
+  return Recip2{hi, __fmul_rn(rem, hi)};
 }
-
+__device__ __forceinline__ float div_rn_recip2(float w, Recip2 y) {
+  return __fmaf_rn(w, y.hi, __fmul_rn(w, y.lo));
+}
 __device__ __forceinline__ bool recip_path_ok(float c) {
   return c >= 7.888609052210118e-31f && c <= 1.2676506002282294e+30f;   // 2^-100 .. 2^100
 }
 
-// Q-A: one group of 256 blocks (16384 weights, 32 KB of bf16) per CTA iteration.  Thread t
-// handles chunk it * 256 + t of the group for it = 0..7 (one 16-byte load each, all eight
-// issued before any is used); the eight lanes of a chunk's block reduce its absmax with
-// three xor shuffles.  Per weight: the correctly rounded n = w / absmax (one reciprocal per
-// block, three fp32 operations per weight), the nearest level, nibble packing.  The group's
-// float64 absmax sum follows the adjacent-pair tree: each warp-iteration covers blocks
-// 4m .. 4m + 3 (m = it * 8 + warp), summed as ((a0 + a1) + (a2 + a3)) by two shuffles, and
-// the 64 four-block sums of the group are reduced by one warp in index order.
-constexpr int kQuantThreads = 256;
-constexpr int kGroupChunks = kB2 * 8;          // 16-byte chunks per group of 256 blocks
+// Q-A: one group of 256 blocks (16384 weights, 32 KB of bf16) per CTA iteration; thread t
+// takes block t of the group: eight 16-byte loads (128 contiguous bytes, all in flight before
+// any is used), absmax over its 64 weights, the correctly rounded n = w / absmax, the nearest
+// level, 32 bytes of packed codes.  The group's float64 sum of its 256 absmax values follows
+// the adjacent-pair tree: the xor butterfly over the 32 lanes of each warp (blocks
+// 32 w .. 32 w + 31), then the eight warp sums in order.
+constexpr int kQuantThreads = kB2;             // one block of 64 weights per thread
 
-__global__ void __launch_bounds__(kQuantThreads) nf4_quant_groups_kernel(const uint16_t* __restrict__ W,
-                                                                         int64_t numel, int64_t ng,
-                                                                         uint32_t* __restrict__ codes32,
-                                                                         float* __restrict__ absmax,
-                                                                         double* __restrict__ gsum) {
+// Codes of a block whose absmax lies outside [2^-100, 2^100] (or of a ragged last block):
+// one correctly rounded division per weight, the weights re-read from W (zero past numel).
+__device__ __noinline__ void codes_by_division(const uint16_t* __restrict__ W, int64_t e0, int64_t numel, float m,
+                                               const BucketEntry (*tab)[32], int lane, uint32_t* __restrict__ dst) {
+  for (int i = 0; i < 8; ++i) {
+    uint32_t p = 0u;
+    for (int j = 0; j < 8; ++j) {
+      const int64_t e = e0 + 8 * i + j;
+      const float w = e < numel ? __uint_as_float((uint32_t)W[e] << 16) : 0.0f;
+      p |= nearest_code(__fdiv_rn(w, m), tab, lane) << (4 * j);
+    }
+    dst[i] = p;
+  }
+}
+
+// The ragged last block (zero-padded past numel), or any block when W holds no whole block:
+// absmax and codes straight from global memory, one correctly rounded division per weight.
+// Returns the block's absmax.
+__device__ __noinline__ float quant_block_global(const uint16_t* __restrict__ W, int64_t b, int64_t numel,
+                                                 const BucketEntry (*tab)[32], int lane, uint32_t* __restrict__ codes32,
+                                                 float* __restrict__ absmax) {
+  const int64_t e0 = b * kB1;
+  float m = 0.0f;
+  for (int64_t e = e0; e < e0 + kB1 && e < numel; ++e) m = fmaxf(m, fabsf(__uint_as_float((uint32_t)W[e] << 16)));
+  absmax[b] = m;
+  if (m > 0.0f) {
+    codes_by_division(W, e0, numel, m, tab, lane, codes32 + b * 8);
+  } else {
+    for (int i = 0; i < 8; ++i) codes32[b * 8 + i] = 0x77777777u;
+  }
+  return m;
+}
+
+// Q-A, streaming form.  Persistent CTAs, two per SM: one thread of the last warp streams
+// groups of 256 blocks (32 KB) into a ring of kQStages shared-memory stages with TMA tile loads
+// of a [blocks][64] bf16 view of W (128-byte swizzle: chunk j of block row r sits at chunk
+// position j ^ (r % 8), so the warps read their blocks without bank conflicts); sixteen
+// warps code the stages in order.  Threads 2r and 2r + 1 own block r of the group, 32
+// weights each: their chunks come from shared memory, then absmax (one shuffle
+// joins the halves), the correctly rounded n = w / absmax, the nearest level and 16 bytes of
+// packed codes each.  The group's float64 absmax sum follows the adjacent-pair tree: the xor
+// butterfly over each warp's 16 blocks, then the sixteen warp sums in order.
+constexpr int kQStages = 3;
+constexpr int kQStageBytes = kB2 * kB1 * 2;           // 32 KB
+constexpr int kQGroupWarps = 16;                      // warps coding one group (two threads per block)
+constexpr int kQConsumerWarps = kQGroupWarps;
+constexpr int kQThreads = 32 * (kQConsumerWarps + 1);
+constexpr int kQSmemBytes = kQStages * kQStageBytes + 1024;
+
+struct QuantParams {
+  CUtensorMap w_map;          // W as [nb_full][64] bf16, box 64 x 256, 128-byte swizzle
+  const uint16_t* W;
+  int64_t numel, nb, nb_full, ng;
+  uint32_t* codes32;
+  float* absmax;
+  double* gsum;
+};
+
+__global__ void __launch_bounds__(kQThreads, 2) nf4_quant_stream_kernel(const __grid_constant__ QuantParams p) {
+  extern __shared__ uint8_t qsmem_dyn[];
+  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(qsmem_dyn) + 1023) & ~uintptr_t(1023));
   __shared__ BucketEntry tab[33][32];
-  __shared__ double sum4[64];
+  __shared__ uint64_t full[kQStages], empty[kQStages];
+  __shared__ double warp_sum[2][kQGroupWarps];
+  __shared__ uint32_t abort_flag;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kQStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kQGroupWarps);
+    }
+    abort_flag = 0u;
+    mbar_fence_init();
+  }
   build_bucket_table(tab);
   __syncthreads();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int64_t nchunks = 8 * ((numel + kB1 - 1) / kB1);   // chunks of whole blocks: the padded tail codes to level 7
-  for (int64_t g = blockIdx.x; g < ng; g += gridDim.x) {
-    const int64_t c0 = g * kGroupChunks + threadIdx.x;
-    uint4 v[8];
-    const bool whole = (g + 1) * kGroupChunks * 8 <= numel;   // every chunk of the group is full
-#pragma unroll
-    for (int it = 0; it < 8; ++it) {
-      const int64_t c = c0 + it * kQuantThreads;
-      if (whole || (c + 1) * 8 <= numel) {
-        v[it] = __ldg(reinterpret_cast<const uint4*>(W) + c);
-      } else {
-        uint32_t u[4] = {0u, 0u, 0u, 0u};
-        for (int i = 0; i < 8; ++i)
-          if (c * 8 + i < numel) u[i >> 1] |= (uint32_t)W[c * 8 + i] << (16 * (i & 1));
-        v[it] = make_uint4(u[0], u[1], u[2], u[3]);
+  volatile uint32_t* abort_word = &abort_flag;
+  const int64_t n_local = p.ng > blockIdx.x ? (p.ng - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+
+  if (warp == kQConsumerWarps) {
+    // ------------------------------------------------------------------ producer
+    if (lane == 0 && p.nb_full > 0) {
+      tma_prefetch_desc(&p.w_map);
+      int64_t issued = 0;
+      for (int64_t i = 0; i < n_local; ++i) {
+        const int s = (int)(i % kQStages);
+        const uint32_t ph = (uint32_t)(i / kQStages) & 1u;
+        if (!mbar_wait_thread(&empty[s], ph ^ 1u, abort_word, kErrWaitEmpty)) break;
+        const int64_t g = blockIdx.x + i * gridDim.x;
+        mbar_arrive_expect_tx(&full[s], kQStageBytes);
+        tma_load_2d(ring + s * kQStageBytes, &p.w_map, 0, (int32_t)(g * kB2), &full[s]);
+        issued = i + 1;
+      }
+      // drain copies still in flight before the CTA's shared memory goes away
+      for (int64_t i = issued > kQStages ? issued - kQStages : 0; i < issued; ++i) {
+        const int s = (int)(i % kQStages);
+        const uint32_t ph = (uint32_t)(i / kQStages) & 1u;
+        for (int k = 0; k < (1 << 22) && !mbar_try_wait(&full[s], ph); ++k) {}
       }
     }
+  } else {
+    // ------------------------------------------------------------------ consumers
+    const int t = threadIdx.x;
+    const int r = t >> 1, h = t & 1;          // block of the group, and which half of it
+    int parity = 0;
+    for (int64_t i = 0; i < n_local; ++i, parity ^= 1) {
+      const int s = (int)(i % kQStages);
+      const uint32_t ph = (uint32_t)(i / kQStages) & 1u;
+      const int64_t g = blockIdx.x + i * gridDim.x;
+      const int64_t b = g * kB2 + r;
+      // a warp whose wait gave up still takes part in the group barrier below, so that the
+      // other warps of its group are not left waiting there; all of them leave after it
+      bool ok = true;
+      uint4 v[4];
+      if (p.nb_full > 0) {
+        ok = mbar_wait(&full[s], ph, abort_word, kErrWaitTma);
+        if (ok) {
+          const uint8_t* row = ring + s * kQStageBytes + r * 128;
 #pragma unroll
-    for (int it = 0; it < 8; ++it) {
-      const int64_t c = c0 + it * kQuantThreads;
-      const uint32_t u[4] = {v[it].x, v[it].y, v[it].z, v[it].w};
-      float w[8];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        w[2 * i] = __uint_as_float(u[i] << 16);
-        w[2 * i + 1] = __uint_as_float(u[i] & 0xFFFF0000u);
-      }
-      float m = 0.0f;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(w[i]));
-      m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-      m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
-      m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
-      // four-block subtree sum of this warp-iteration (lanes 0, 8, 16, 24 hold blocks 4m..4m+3)
-      double s = (double)m;
-      s = s + __shfl_xor_sync(0xFFFFFFFFu, s, 8);
-      s = s + __shfl_xor_sync(0xFFFFFFFFu, s, 16);
-      if (lane == 0) sum4[it * 8 + warp] = s;
-      if (c >= nchunks) continue;
-      if ((lane & 7) == 0) absmax[c >> 3] = m;
-      uint32_t packed = 0x77777777u;             // all-zero block: every weight is level 7
-      if (m > 0.0f) {
-        packed = 0u;
-        if (recip_path_ok(m)) {
-          const float y = __frcp_rn(m);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) packed |= nearest_code(div_rn_by_recip(w[i], m, y), tab, lane) << (4 * i);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) packed |= nearest_code(__fdiv_rn(w[i], m), tab, lane) << (4 * i);
+          for (int j = 0; j < 4; ++j) v[j] = *reinterpret_cast<const uint4*>(row + (((4 * h + j) ^ (r & 7)) << 4));
         }
       }
-      codes32[c] = packed;
-    }
-    __syncthreads();
-    if (warp == 0) {
-      double t = sum4[2 * lane] + sum4[2 * lane + 1];
+      const bool whole = ok && b < p.nb_full;
+      float m = 0.0f;
+      if (ok && p.nb_full > 0) {
+        // every loaded word enters the absmax, so the stage's data are in registers before the
+        // stage is handed back for the next load
 #pragma unroll
-      for (int off = 1; off < 32; off <<= 1) t = t + __shfl_xor_sync(0xFFFFFFFFu, t, off);
-      if (lane == 0) gsum[g] = t;
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t u[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            m = fmaxf(m, fabsf(__uint_as_float(u[k] << 16)));
+            m = fmaxf(m, fabsf(__uint_as_float(u[k] & 0xFFFF0000u)));
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+        if (!whole) m = 0.0f;
+      }
+      if (!whole && ok && b < p.nb && h == 0) {
+        m = quant_block_global(p.W, b, p.numel, tab, lane, p.codes32, p.absmax);
+      }
+      m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));   // join the two halves of each block
+      double sum = (double)m;
+#pragma unroll
+      for (int off = 2; off < 32; off <<= 1) sum = sum + __shfl_xor_sync(0xFFFFFFFFu, sum, off);
+      if (lane == 0) warp_sum[parity][warp] = sum;
+      if (whole) {
+        if (h == 0) p.absmax[b] = m;
+        uint4* dst = reinterpret_cast<uint4*>(p.codes32 + b * 8) + h;
+        if (m > 0.0f && recip_path_ok(m)) {
+          const Recip2 y = recip2(m);
+          uint32_t packed[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t u[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+            uint32_t pk = 0u;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              pk += nearest_code(div_rn_recip2(__uint_as_float(u[k] << 16), y), tab, lane) << (8 * k);
+              pk += nearest_code(div_rn_recip2(__uint_as_float(u[k] & 0xFFFF0000u), y), tab, lane) << (8 * k + 4);
+            }
+            packed[j] = pk;
+          }
+          *dst = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        } else if (m > 0.0f) {
+          if (h == 0) codes_by_division(p.W, b * kB1, p.numel, m, tab, lane, p.codes32 + b * 8);
+        } else {
+          *dst = make_uint4(0x77777777u, 0x77777777u, 0x77777777u, 0x77777777u);   // all-zero block: level 7
+        }
+      }
+      // one barrier of the group's warps per group: the warp sums alternate between two
+      // buffers, so thread 0 reads this group's while the warps fill the other one
+      asm volatile("bar.sync 1, %0;" ::"r"(32 * kQGroupWarps) : "memory");
+      if (*abort_word) break;
+      if (t == 0) {
+        const double* w = warp_sum[parity];
+        const double q0 = ((w[0] + w[1]) + (w[2] + w[3])) + ((w[4] + w[5]) + (w[6] + w[7]));
+        const double q1 = ((w[8] + w[9]) + (w[10] + w[11])) + ((w[12] + w[13]) + (w[14] + w[15]));
+        p.gsum[g] = q0 + q1;
+      }
     }
-    __syncthreads();
   }
   // let the dependent double-quantization kernel start its launch while this grid drains
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -183,6 +299,22 @@ __global__ void __launch_bounds__(256) dq_mean_groups_kernel(const float* __rest
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   // the quantize kernel's absmax values and group sums are complete and visible after this
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  // this warp's first group: its absmax values are in flight while the mean is formed
+  int64_t g = (int64_t)blockIdx.x * 8 + warp;
+  float a[8];
+  auto load_group = [&](int64_t gg) {
+    const int64_t b0 = gg * kB2 + lane * 8;
+    if (b0 + 8 <= nb) {
+      const float4* src = reinterpret_cast<const float4*>(absmax + b0);
+      const float4 x0 = src[0], x1 = src[1];
+      a[0] = x0.x; a[1] = x0.y; a[2] = x0.z; a[3] = x0.w;
+      a[4] = x1.x; a[5] = x1.y; a[6] = x1.z; a[7] = x1.w;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) a[i] = (b0 + i < nb) ? absmax[b0 + i] : 0.0f;
+    }
+  };
+  if (g < ng) load_group(g);
   const int64_t nchunks = (ng + 2047) / 2048;
   for (int64_t ch = 0; ch < nchunks; ++ch) {
     const int64_t i0 = ch * 2048 + 8 * (int64_t)threadIdx.x;
@@ -223,15 +355,16 @@ __global__ void __launch_bounds__(256) dq_mean_groups_kernel(const float* __rest
     mean = __double2float_rn(warp_sum[0] / (double)nb);
   }
   if (blockIdx.x == 0 && threadIdx.x == 0) mean_out[0] = mean;
-  for (int64_t g = (int64_t)blockIdx.x * 8 + warp; g < ng; g += (int64_t)gridDim.x * 8) {
+  for (; g < ng; g += (int64_t)gridDim.x * 8) {
     float d[8];
     float m = 0.0f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int64_t b = g * kB2 + lane * 8 + i;
-      d[i] = (b < nb) ? __fsub_rn(absmax[b], mean) : 0.0f;
+      d[i] = (b < nb) ? __fsub_rn(a[i], mean) : 0.0f;
       m = fmaxf(m, fabsf(d[i]));
     }
+    if (g + (int64_t)gridDim.x * 8 < ng) load_group(g + (int64_t)gridDim.x * 8);
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
     uint32_t e[8];
@@ -344,21 +477,31 @@ static int grid_for(int64_t threads, int per_block, int cap) {
   return (int)g;
 }
 
-cudaError_t launch_quantize(const uint16_t* W, int64_t numel, uint8_t* codes, uint8_t* scale_codes, float* c2,
-                            float* mean, float* absmax_ws, double* gsum_ws, cudaStream_t st, int sw_encode) {
+cudaError_t launch_quantize(const CUtensorMap* w_map, const uint16_t* W, int64_t numel, uint8_t* codes,
+                            uint8_t* scale_codes, float* c2, float* mean, float* absmax_ws, double* gsum_ws,
+                            cudaStream_t st, int sw_encode) {
   const int64_t nb = (numel + kB1 - 1) / kB1;
   const int64_t ng = (nb + kB2 - 1) / kB2;
   if (ng > (int64_t)kMaxMeanChunks * 2048) return cudaErrorInvalidValue;
-  int sms = 148, per_sm = 4;
+  int sms = 148;
   int dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // a grid-stride loop over groups: as many CTAs as fit on the device at once
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, nf4_quant_groups_kernel, kQuantThreads, 0) != cudaSuccess ||
-      per_sm < 1)
-    per_sm = 1;
-  nf4_quant_groups_kernel<<<grid_for(ng, 1, sms * per_sm), kQuantThreads, 0, st>>>(
-      W, numel, ng, reinterpret_cast<uint32_t*>(codes), absmax_ws, gsum_ws);
-  cudaError_t e = cudaGetLastError();
+  static std::atomic<uint64_t> configured{0};
+  cudaError_t e = enable_smem_once(nf4_quant_stream_kernel, kQSmemBytes, configured);
+  if (e != cudaSuccess) return e;
+  QuantParams qp;
+  memset(&qp, 0, sizeof(qp));
+  if (w_map) qp.w_map = *w_map;
+  qp.W = W;
+  qp.numel = numel;
+  qp.nb = nb;
+  qp.nb_full = w_map ? numel / kB1 : 0;
+  qp.ng = ng;
+  qp.codes32 = reinterpret_cast<uint32_t*>(codes);
+  qp.absmax = absmax_ws;
+  qp.gsum = gsum_ws;
+  nf4_quant_stream_kernel<<<grid_for(ng, 1, 2 * sms), kQThreads, kQSmemBytes, st>>>(qp);
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   // The double-quantization kernel may launch while the quantize grid drains (programmatic
   // dependent launch); it waits for that grid's results before reading them.

@@ -2,12 +2,16 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 namespace qnf4 {
 
-cudaError_t launch_quantize(const uint16_t* W, int64_t numel, uint8_t* codes, uint8_t* scale_codes, float* c2,
-                            float* mean, float* absmax_ws, double* gsum_ws, cudaStream_t st, int sw_encode);
+// w_map: W viewed as [numel / 64][64] bf16 (box 64 x 256, 128-byte swizzle), or NULL when
+// numel < 64 (no whole block).
+cudaError_t launch_quantize(const CUtensorMap* w_map, const uint16_t* W, int64_t numel, uint8_t* codes,
+                            uint8_t* scale_codes, float* c2, float* mean, float* absmax_ws, double* gsum_ws,
+                            cudaStream_t st, int sw_encode);
 cudaError_t launch_dequant(const uint8_t* codes, const uint8_t* scale_codes, const float* c2, const float* mean,
                            int64_t numel, uint16_t* out, cudaStream_t st);
 cudaError_t launch_e4m3_encode(const float* v, int64_t n, uint8_t* out, int sw, cudaStream_t st);

@@ -402,7 +402,11 @@ int nf4_quantize_dq(const uint16_t* W, int64_t numel, uint8_t* codes, uint8_t* s
   const int64_t nb = (numel + 63) / 64;
   float* absmax = static_cast<float*>(workspace);
   double* gsum = reinterpret_cast<double*>(static_cast<char*>(workspace) + align_up((size_t)nb * 4, 256));
-  cudaError_t e = qnf4::launch_quantize(W, numel, codes, scale_codes, c2, mean, absmax, gsum,
+  CUtensorMap wmap;
+  const bool has_map = numel >= 64;
+  if (has_map)
+    if (int rc = make_map(&wmap, W, true, 64, (uint64_t)(numel / 64), 128, 64, 256)) return rc;
+  cudaError_t e = qnf4::launch_quantize(has_map ? &wmap : nullptr, W, numel, codes, scale_codes, c2, mean, absmax, gsum,
                                         static_cast<cudaStream_t>(stream), 0);
   if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
   return QNF4_OK;
@@ -426,7 +430,11 @@ int nf4_quantize_dq_noalloc(const uint16_t* W, int64_t numel, uint8_t* codes, ui
   const int64_t nb = (numel + 63) / 64;
   float* absmax = static_cast<float*>(scratch);
   double* gsum = reinterpret_cast<double*>(static_cast<char*>(scratch) + align_up((size_t)nb * 4, 256));
-  cudaError_t e = qnf4::launch_quantize(W, numel, codes, scale_codes, c2, mean, absmax, gsum,
+  CUtensorMap wmap;
+  const bool has_map = numel >= 64;
+  if (has_map)
+    if (int rc = make_map(&wmap, W, true, 64, (uint64_t)(numel / 64), 128, 64, 256)) return rc;
+  cudaError_t e = qnf4::launch_quantize(has_map ? &wmap : nullptr, W, numel, codes, scale_codes, c2, mean, absmax, gsum,
                                         static_cast<cudaStream_t>(stream), 0);
   if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
   return QNF4_OK;
