@@ -23,7 +23,7 @@ namespace qnf4 {
 // of them.  code = (#midpoints below the bucket) + (n > the bucket's midpoint).  The
 // midpoint test uses theta_j = the largest fp32 not above the exact midpoint, which makes
 // n > theta_j equivalent to n > midpoint for every fp32 n (ties go to the lower level).
-struct BucketEntry {
+struct __align__(8) BucketEntry {
   uint32_t base;
   float thr;
 };
