@@ -4,8 +4,7 @@
 // The 128-row A side is either loaded by TMA or produced on chip from packed NF4 codes; the
 // dequantized 16-bit weights exist only in shared memory or, with A_TMEM, in tensor memory,
 // never in HBM.  The B side is a K-major bf16 tile loaded by TMA.  Lane 0 of warp 1 issues
-// tcgen05.mma (kind::f16, bf16 x bf16 -> fp32) into the TMEM accumulator; the eight producer
-// warps read it back for the epilogue.
+// tcgen05.mma (kind::f16, bf16 x bf16 -> fp32) into the TMEM accumulator.
 //
 // The method's forward and backward ("QLoRA Paper Breakdown: 4-Bit NormalFloat (NF4), Double
 // Quantization, and Paged Optimizers" (fullstackaihub), section 4) use this engine for
@@ -15,14 +14,21 @@
 // parts, run as extra k-blocks of the same accumulator, so that the adapter terms keep close
 // to fp32 accuracy through bf16 tensor-core inputs.
 //
-// Warp roles: warps 0 and 10.. (kTmaWarps of them) issue the TMA loads of alternate k-blocks,
-// warp 1 allocates TMEM and (lane 0) issues the MMAs, warps 2-9 run the dequant producer (two
-// groups of four warps on alternate k-blocks) and then the epilogue (each group drains half of
-// the accumulator columns).  Per pipeline stage s:
+// The kernel is persistent: one CTA per SM walks the tiles blockIdx.x, blockIdx.x + gridDim.x,
+// ... (row tiles fastest).  Ring stages and their phases are counted over the CTA's whole
+// sequence of k-blocks, so the loads and the dequant production of the next tile proceed
+// while the current one finishes.  Warp roles: warps 0 and 10 issue the TMA loads of
+// alternate k-blocks, warp 1 allocates TMEM and (lane 0) issues the MMAs, warps 2-9 run the
+// dequant producer (two groups of four warps on alternate k-blocks), warps 11.. drain the
+// accumulator (the epilogue).  With A in shared memory the accumulator is double-buffered in
+// TMEM, so a tile's epilogue overlaps the next tile's MMAs; with A in TMEM (which then holds
+// the A slots beside one accumulator) eight epilogue warps drain it, and the next tile's
+// MMAs start once they are done.  Per stage s:
 //   full[s]   the B tile (and a TMA-loaded A tile) has landed;
 //   cfull[s]  the codes have landed (shared-memory A), or a plain arrive: producers may start;
 //   prod[s]   the producers wrote the A tile, after they also saw full[s];
-//   empty[s]  the MMAs that read stage s completed (tcgen05.commit).
+//   empty[s]  the MMAs that read stage s completed (tcgen05.commit);
+// per accumulator buffer b: accfull[b] (its MMAs completed), accempty[b] (drained).
 #pragma once
 
 #include "nf4_device.cuh"
@@ -34,9 +40,9 @@ constexpr int kBM = 128;
 constexpr int kBK = 64;
 // A bulk-tensor load holds the thread that issues it for a few hundred cycles, whatever the box
 // size, while loads from different warps proceed side by side: kTmaWarps warps share the loads,
-// warp w (warp 0, then warps 10, 11, ...) taking the k-blocks it with it % kTmaWarps == w.
+// warp w (warp 0, then warp 10) taking the k-blocks whose global index i has i % kTmaWarps == w.
 constexpr int kTmaWarps = 2;
-constexpr int kThreads = 320 + 32 * (kTmaWarps - 1);   // + MMA warp, two groups of four producer / epilogue warps
+constexpr int kEpiWarp0 = 11;       // first epilogue warp
 constexpr int kCodesBytes = 4096;   // packed codes of one 128 x 64 weight tile
 
 // A_TMEM: the A tile lives in tensor memory (slot s at column kATmemCol0 + 32 s), so a stage
@@ -53,13 +59,20 @@ struct Cfg {
   // stages and wait on every phase of their barriers (a parity wait that skips a phase can
   // pass early).
   static constexpr int kStages = (kStagesRaw > 8 ? 8 : kStagesRaw) & ~1;
-  static constexpr int kTmemCols = A_TMEM ? 512 : (BN <= 32 ? 32 : BN);
+  // Accumulator buffers: two when TMEM has room (A in shared memory), else one.
+  static constexpr int kAccBufs = A_TMEM ? 1 : 2;
+  static constexpr int kEpiWarps = A_TMEM ? 8 : 4;
+  static constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
+  // accumulator buffer b starts at TMEM column b * kAccStride (at least 32 columns apart)
+  static constexpr int kAccStride = BN < 32 ? 32 : BN;
+  static constexpr int kTmemCols = A_TMEM ? 512 : 2 * kAccStride;
   static_assert(!A_TMEM || (BN == 256 && kStages <= 8), "A in TMEM: 256-column accumulator + 8 slots of 32 columns");
   static constexpr int kBarrierBytes = 512;
   static constexpr int kSmemBytes = kStages * kStageBytes + kBarrierBytes + 1024;
   static_assert(kStages >= 2 && kStages % 2 == 0, "pipeline too shallow, or odd");
   static_assert(kStages % kTmaWarps == 0, "each TMA warp must own whole stages");
   static_assert(kBBytes % 1024 == 0, "B tile must keep 1024-byte alignment");
+  static_assert(4 * kStages * 8 + 5 * 8 + 8 <= kBarrierBytes, "barrier area");
 };
 
 struct IterPos {
@@ -234,29 +247,107 @@ __device__ __noinline__ void umma_kblock_ragged(uint32_t tmem_acc, uint32_t a_ad
   }
 }
 
+// One tile of the persistent schedule: tile t -> (row tile, column tile, K split), row tiles
+// fastest; its k-block range of segment 0 and its number of k-blocks (later segments run in
+// split 0 only).
+struct TileInfo {
+  int row0, col0, split, kb_begin, kb_end, n_iters;
+};
+
+template <int BN>
+__device__ __forceinline__ TileInfo tile_info(const GemmParams& p, int tiles_m, int tiles_n, int64_t t) {
+  TileInfo ti;
+  const int64_t per_split = (int64_t)tiles_m * tiles_n;
+  ti.split = (int)(t / per_split);
+  const int64_t rem = t - (int64_t)ti.split * per_split;
+  ti.row0 = (int)(rem % tiles_m) * kBM;
+  ti.col0 = (int)(rem / tiles_m) * BN;
+  ti.kb_begin = ti.split * p.kb_per_split;
+  ti.kb_end = ti.kb_begin + p.kb_per_split;
+  if (ti.kb_end > p.seg[0].kblocks) ti.kb_end = p.seg[0].kblocks;
+  ti.n_iters = ti.kb_end - ti.kb_begin;
+  if (ti.split == 0)
+    for (int s = 1; s < p.nseg; ++s) ti.n_iters += p.seg[s].kblocks;
+  return ti;
+}
+
+// Walks this CTA's k-blocks (tile by tile) in steps of 1 or 2 from `first`; stage and phase
+// are the ring position of the current k-block, counted over the CTA's whole sequence (32-bit
+// and incremental: they sit on the issuing threads' critical path).
+template <int BN, int S>
+struct KIter {
+  int tiles_m, tiles_n;
+  int64_t ntiles, t;
+  TileInfo ti;
+  int it;
+  int stage;
+  uint32_t phase;
+  bool done;
+
+  __device__ __forceinline__ void init(const GemmParams& p, int first) {
+    tiles_m = (p.rows + kBM - 1) / kBM;
+    tiles_n = (p.cols + BN - 1) / BN;
+    ntiles = (int64_t)tiles_m * tiles_n * p.splits;
+    t = blockIdx.x;
+    done = t >= ntiles;
+    it = 0;
+    stage = 0;
+    phase = 0u;
+    if (!done) ti = tile_info<BN>(p, tiles_m, tiles_n, t);
+    advance(p, first);
+  }
+  __device__ __forceinline__ void advance(const GemmParams& p, int k) {
+    it += k;
+    stage += k;
+    if (stage >= S) {
+      stage -= S;
+      phase ^= 1u;
+    }
+    while (!done && it >= ti.n_iters) {
+      it -= ti.n_iters;
+      t += gridDim.x;
+      if (t >= ntiles) {
+        done = true;
+      } else {
+        ti = tile_info<BN>(p, tiles_m, tiles_n, t);
+      }
+    }
+  }
+};
+
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+// TMA tile load with an L2 cache-eviction hint (no multicast).
+__device__ __forceinline__ void tma_load_2d_hint(void* smem_dst, const CUtensorMap* map, int32_t x, int32_t y,
+                                                 uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, "
+      "{%2, %3}], [%4], %5;" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
 template <int BN, bool GENERIC, bool A_TMEM>
-__global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_constant__ GemmParams p) {
+__global__ void __launch_bounds__(Cfg<BN, A_TMEM>::kThreads, 1) qlora_gemm_kernel(const __grid_constant__ GemmParams p) {
   using C = Cfg<BN, A_TMEM>;
   constexpr int S = C::kStages;
+  constexpr int NB = C::kAccBufs;
   extern __shared__ uint8_t smem_dyn[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
   uint64_t* cfull = full + S;   // the stage's codes have landed (or a plain arrive): producers may start
   uint64_t* prod = cfull + S;
   uint64_t* empty = prod + S;
-  uint64_t* accfull = empty + S;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accfull + 1);
+  uint64_t* accfull = empty + S;      // [2]
+  uint64_t* accempty = accfull + 2;   // [2]
+  uint64_t* mma_done = accempty + 2;  // the MMA thread's final commit
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile uint32_t* abort_word = tmem_slot + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row0 = blockIdx.x * kBM, col0 = blockIdx.y * BN, split = blockIdx.z;
-  const int kb_begin = split * p.kb_per_split;
-  int kb_end = kb_begin + p.kb_per_split;
-  if (kb_end > p.seg[0].kblocks) kb_end = p.seg[0].kblocks;
-  const bool first_split = (split == 0);
-  int n_iters = kb_end - kb_begin;
-  if (first_split)
-    for (int s = 1; s < p.nseg; ++s) n_iters += p.seg[s].kblocks;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -265,7 +356,11 @@ __global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_co
       mbar_init(&prod[s], 4);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(accfull, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&accfull[b], 1);
+      mbar_init(&accempty[b], C::kEpiWarps);
+    }
+    mbar_init(mma_done, 1);
     *abort_word = 0u;
     mbar_fence_init();
   }
@@ -279,52 +374,55 @@ __global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_co
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem_acc = *tmem_slot;
+  const uint32_t tmem_base = *tmem_slot;
 
   auto stage_a = [&](int s) { return smem + s * C::kStageBytes; };
   auto stage_b = [&](int s) { return smem + s * C::kStageBytes + C::kABytes; };
   auto stage_c = [&](int s) { return smem + s * C::kStageBytes + C::kABytes + C::kBBytes; };
 
-  if (warp == 0 || warp >= 10) {
+  if (warp == 0 || warp == 10) {
     // ------------------------------------------------------------------ TMA producers
-    const int tw = (warp == 0) ? 0 : warp - 9;
-    int last_issue[8];
+    const int tw = (warp == 0) ? 0 : 1;
+    const uint64_t codes_policy = l2_policy_evict_last();   // the codes are re-read by every column tile
+    int last_issue[8];            // phase of the last load issued into each stage (-1: none)
     for (int s = 0; s < 8; ++s) last_issue[s] = -1;
     bool ok = true;
-    for (int it = tw; it < n_iters && ok; it += kTmaWarps) {
-      const int s = it % S;
-      const uint32_t ph = (uint32_t)(it / S) & 1u;
+    KIter<BN, S> ki;
+    ki.init(p, tw);
+    for (; !ki.done; ki.advance(p, kTmaWarps)) {
+      const int s = ki.stage;
+      const uint32_t ph = ki.phase;
       if (!mbar_wait(&empty[s], ph ^ 1u, abort_word, kErrWaitEmpty)) { ok = false; break; }
-      const IterPos ip = iter_pos(p, it, kb_begin, kb_end, first_split);
+      const IterPos ip = iter_pos(p, ki.it, ki.ti.kb_begin, ki.ti.kb_end, ki.ti.split == 0);
       const GemmSeg& sg = p.seg[ip.seg];
       const bool nf4 = (sg.a_src == kANf4K || sg.a_src == kANf4MN);
       if (lane == 0) {
         // With A in shared memory the codes complete on cfull[s], so the producers can
         // dequantize while the (larger) B tile is still landing on full[s].  With A in tensor
-        // memory (6 stages) that gains nothing and the codes complete on full[s].
+        // memory the codes complete on full[s].
         const bool codes_tma = nf4 && !GENERIC;
         mbar_arrive_expect_tx(&full[s], C::kBBytes + (nf4 ? 0u : (uint32_t)C::kABytes) +
                                             ((A_TMEM && codes_tma) ? (uint32_t)kCodesBytes : 0u));
         if (!A_TMEM && codes_tma) mbar_arrive_expect_tx(&cfull[s], kCodesBytes);
         else mbar_arrive(&cfull[s]);
-        last_issue[s] = it;
+        last_issue[s] = (int)ph;
       }
       __syncwarp();
-      // A bulk-tensor load holds its issuing thread for a few hundred cycles whatever the box
-      // size, so one thread issuing the k-block's two or three loads one after the other
-      // would pace the whole pipeline.  Lanes 0..2 each take one load and issue them as a
-      // single instruction: lane 0 the B tile, lanes 1 and 2 the A side.
+      // Lanes 0..2 each take one load and issue them as a single instruction: lane 0 the B
+      // tile, lanes 1 and 2 the A side.
+      const int row0 = ki.ti.row0, col0 = ki.ti.col0;
       const int k = sg.a_k0 + ip.kb * kBK;
       int map = -1, cx = 0, cy = 0;
+      bool codes = false;
       uint8_t* dst = nullptr;
       uint64_t* bar = &full[s];
       if (lane == 0) {
         map = sg.b_map; dst = stage_b(s); cx = sg.b_k0 + ip.kb * kBK; cy = col0;
       } else if (lane == 1) {
         if (sg.a_src == kANf4K) {
-          if (!GENERIC) { map = sg.a_map; dst = stage_c(s); cx = k / 2; cy = row0; bar = A_TMEM ? &full[s] : &cfull[s]; }
+          if (!GENERIC) { map = sg.a_map; dst = stage_c(s); cx = k / 2; cy = row0; bar = A_TMEM ? &full[s] : &cfull[s]; codes = true; }
         } else if (sg.a_src == kANf4MN) {
-          if (!GENERIC) { map = sg.a_map; dst = stage_c(s); cx = row0 / 2; cy = k; bar = A_TMEM ? &full[s] : &cfull[s]; }
+          if (!GENERIC) { map = sg.a_map; dst = stage_c(s); cx = row0 / 2; cy = k; bar = A_TMEM ? &full[s] : &cfull[s]; codes = true; }
         } else if (sg.a_src == kATmaK) {
           if (!A_TMEM) { map = sg.a_map; dst = stage_a(s); cx = k; cy = row0; }
         } else {
@@ -333,14 +431,17 @@ __global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_co
       } else if (lane == 2 && sg.a_src == kATmaMN) {
         map = sg.a_map; dst = stage_a(s) + 8192; cx = row0 + 64; cy = k;
       }
-      if (map >= 0) tma_load_2d(dst, &p.maps[map], cx, cy, bar);
+      if (map >= 0) {
+        if (codes) tma_load_2d_hint(dst, &p.maps[map], cx, cy, bar, codes_policy);
+        else tma_load_2d(dst, &p.maps[map], cx, cy, bar);
+      }
       __syncwarp();
     }
     if (!ok && lane == 0) {
       // drain copies still in flight before the CTA's shared memory goes away
       for (int s = 0; s < S; ++s)
         if (last_issue[s] >= 0) {
-          const uint32_t ph = (uint32_t)(last_issue[s] / S) & 1u;
+          const uint32_t ph = (uint32_t)last_issue[s];
           for (int i = 0; i < (1 << 20) && !mbar_try_wait(&full[s], ph); ++i) {}
           for (int i = 0; i < (1 << 20) && !mbar_try_wait(&cfull[s], ph); ++i) {}
         }
@@ -357,63 +458,87 @@ __global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_co
     if (lane == 0) {
       uint64_t* const ready = p.has_nf4 ? prod : full;
       const uint32_t ready_err = p.has_nf4 ? kErrWaitProducer : kErrWaitTma;
-      for (int it = 0; it < n_iters; ++it) {
-        const int s = it % S;
-        const uint32_t ph = (uint32_t)(it / S) & 1u;
-        if (!mbar_wait_thread(&ready[s], ph, abort_word, ready_err)) break;
+      const int tiles_m = (p.rows + kBM - 1) / kBM;
+      const int tiles_n = (p.cols + BN - 1) / BN;
+      const int64_t ntiles = (int64_t)tiles_m * tiles_n * p.splits;
+      int s = 0;
+      uint32_t ph = 0u;
+      int64_t tc = 0;           // tiles started
+      bool ok = true;
+      for (int64_t tt = blockIdx.x; tt < ntiles && ok; tt += gridDim.x, ++tc) {
+        const TileInfo ti = tile_info<BN>(p, tiles_m, tiles_n, tt);
+        const int buf = (int)(tc % NB);
+        const uint32_t use = (uint32_t)(tc / NB) & 1u;
+        if (!mbar_wait_thread(&accempty[buf], use ^ 1u, abort_word, kErrWaitMma)) { ok = false; break; }
         tc_fence_after();
-        const IterPos ip = iter_pos(p, it, kb_begin, kb_end, first_split);
-        const GemmSeg& sg = p.seg[ip.seg];
-        const bool a_mn = (sg.a_src == kANf4MN || sg.a_src == kATmaMN);
-        const uint32_t a_addr = smem_u32(stage_a(s));
-        const uint32_t b_addr = smem_u32(stage_b(s));
-        const uint32_t acc = it > 0 ? 1u : 0u;
-        if constexpr (A_TMEM) {
-          (void)a_mn; (void)a_addr;
-          umma_kblock_ts<BN>(tmem_acc, tmem_acc + kATmemCol0 + 32u * (uint32_t)s, b_addr, acc,
-                             ip.last ? sg.k16_last : 4);
-        } else if (!ip.last || sg.k16_last == 4) {
-          if (a_mn) umma_kblock<BN, true>(tmem_acc, a_addr, b_addr, acc);
-          else umma_kblock<BN, false>(tmem_acc, a_addr, b_addr, acc);
-        } else {
-          umma_kblock_ragged<BN>(tmem_acc, a_addr, b_addr, acc, a_mn, sg.k16_last);
+        const uint32_t tmem_acc = tmem_base + (uint32_t)(buf * C::kAccStride);
+        const bool first_split = ti.split == 0;
+        for (int it = 0; it < ti.n_iters; ++it) {
+          if (!mbar_wait_thread(&ready[s], ph, abort_word, ready_err)) { ok = false; break; }
+          tc_fence_after();
+          const IterPos ip = iter_pos(p, it, ti.kb_begin, ti.kb_end, first_split);
+          const GemmSeg& sg = p.seg[ip.seg];
+          const bool a_mn = (sg.a_src == kANf4MN || sg.a_src == kATmaMN);
+          const uint32_t a_addr = smem_u32(stage_a(s));
+          const uint32_t b_addr = smem_u32(stage_b(s));
+          const uint32_t acc = it > 0 ? 1u : 0u;
+          if constexpr (A_TMEM) {
+            (void)a_mn; (void)a_addr;
+            umma_kblock_ts<BN>(tmem_acc, tmem_base + kATmemCol0 + 32u * (uint32_t)s, b_addr, acc,
+                               ip.last ? sg.k16_last : 4);
+          } else if (!ip.last || sg.k16_last == 4) {
+            if (a_mn) umma_kblock<BN, true>(tmem_acc, a_addr, b_addr, acc);
+            else umma_kblock<BN, false>(tmem_acc, a_addr, b_addr, acc);
+          } else {
+            umma_kblock_ragged<BN>(tmem_acc, a_addr, b_addr, acc, a_mn, sg.k16_last);
+          }
+          umma_commit(&empty[s]);
+          if (++s == S) {
+            s = 0;
+            ph ^= 1u;
+          }
         }
-        umma_commit(&empty[s]);
+        if (ok) umma_commit(&accfull[buf]);
       }
-      umma_commit(accfull);   // also on abort: lets the epilogue wait out in-flight MMAs
+      // every MMA issued so far has completed before TMEM is released
+      umma_commit(mma_done);
+      for (int i = 0; i < (1 << 22) && !mbar_try_wait(mma_done, 0u); ++i) {}
     }
     __syncwarp();
-  } else {
+  } else if (warp < kEpiWarp0) {
     // ------------------------------------------------------------------ dequant producer
     // Two groups of four warps take alternate k-blocks; within a group thread t owns one
     // 64-weight unit per k-block.
     const int grp = (warp - 2) >> 2;          // 0: warps 2-5, 1: warps 6-9
     const int t = 32 * (warp & 3) + lane;       // tile row t = TMEM lane t (warp w reaches lanes 32 (w % 4) ..)
-    bool ok = true;
     if (p.has_nf4) {
       const float mean = __ldg(p.mean);
       const int64_t nb = (p.nw * p.kw + kB1 - 1) / kB1;
-      auto geom = [&](int it, bool& nf4, UnitGeom& u) {
-        const IterPos ip = iter_pos(p, it, kb_begin, kb_end, first_split);
+      auto geom = [&](const KIter<BN, S>& q, bool& nf4, UnitGeom& u) {
+        const IterPos ip = iter_pos(p, q.it, q.ti.kb_begin, q.ti.kb_end, q.ti.split == 0);
         const GemmSeg& sg = p.seg[ip.seg];
         nf4 = (sg.a_src == kANf4K || sg.a_src == kANf4MN);
-        if (nf4) u = unit_geom(sg.a_src, t, row0, (int64_t)sg.a_k0 + (int64_t)ip.kb * kBK);
+        if (nf4) u = unit_geom(sg.a_src, t, q.ti.row0, (int64_t)sg.a_k0 + (int64_t)ip.kb * kBK);
       };
+      KIter<BN, S> cur;
+      cur.init(p, grp);
+      KIter<BN, S> nxt = cur;
       bool nf4_next = false;
       UnitGeom u_next{};
       UnitScale sc_next{};
-      if (grp < n_iters) {
-        geom(grp, nf4_next, u_next);
+      if (!nxt.done) {
+        geom(nxt, nf4_next, u_next);
         if (nf4_next) sc_next = fetch_scale<GENERIC>(p, u_next, nb);
       }
-      for (int it = grp; it < n_iters; it += 2) {
-        const int s = it % S;
-        const uint32_t ph = (uint32_t)(it / S) & 1u;
+      for (; !cur.done; cur.advance(p, 2)) {
+        const int s = cur.stage;
+        const uint32_t ph = cur.phase;
         const bool nf4 = nf4_next;
         const UnitGeom u = u_next;
         const UnitScale sc = sc_next;
-        if (it + 2 < n_iters) {               // prefetch the next iteration's scales
-          geom(it + 2, nf4_next, u_next);
+        nxt.advance(p, 2);                    // prefetch the next k-block's scales
+        if (!nxt.done) {
+          geom(nxt, nf4_next, u_next);
           if (nf4_next) sc_next = fetch_scale<GENERIC>(p, u_next, nb);
         }
         Nf4Lut L0, L1;
@@ -427,10 +552,10 @@ __global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_co
             for (int j = 0; j < 8; ++j) words[j] = (j < sc.valid) ? __ldg(src + j) : 0u;
           }
         }
-        if (!mbar_wait(A_TMEM ? &full[s] : &cfull[s], ph, abort_word, kErrWaitTma)) { ok = false; break; }
+        if (!mbar_wait(A_TMEM ? &full[s] : &cfull[s], ph, abort_word, kErrWaitTma)) break;
         if constexpr (A_TMEM) {
           // Row t of the A tile (64 bf16 = 32 columns) into TMEM slot s.  Slot s is free: full[s]
-          // of this iteration follows the release of stage s by the MMAs that last read it.
+          // of this k-block follows the release of stage s by the MMAs that last read it.
           uint32_t v[32];
           if (nf4) {
             if constexpr (!GENERIC) {
@@ -447,8 +572,8 @@ __global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_co
             }
           } else {
             // a kATmaK stretch: row t of the adapter matrix, k-block kb, from global memory
-            const IterPos ip = iter_pos(p, it, kb_begin, kb_end, first_split);
-            const int64_t row = (int64_t)row0 + t;
+            const IterPos ip = iter_pos(p, cur.it, cur.ti.kb_begin, cur.ti.kb_end, cur.ti.split == 0);
+            const int64_t row = (int64_t)cur.ti.row0 + t;
             const int64_t kk = (int64_t)p.seg[ip.seg].a_k0 + (int64_t)ip.kb * kBK;
             const uint4* src = reinterpret_cast<const uint4*>(p.a_glob + row * p.a_glob_ld + kk);
 #pragma unroll
@@ -458,7 +583,7 @@ __global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_co
               v[4 * q] = w4.x; v[4 * q + 1] = w4.y; v[4 * q + 2] = w4.z; v[4 * q + 3] = w4.w;
             }
           }
-          tmem_st_32x32b_x32(tmem_acc + ((uint32_t)(32 * (warp & 3)) << 16) + kATmemCol0 + 32u * (uint32_t)s, v);
+          tmem_st_32x32b_x32(tmem_base + ((uint32_t)(32 * (warp & 3)) << 16) + kATmemCol0 + 32u * (uint32_t)s, v);
           tmem_st_wait();
           tc_fence_before();
         } else if (nf4) {
@@ -485,53 +610,72 @@ __global__ void __launch_bounds__(kThreads, 1) qlora_gemm_kernel(const __grid_co
           fence_proxy_async_smem();
         }
         // prod[s] is the MMA issuer's only wait, so it also vouches for the B tile
-        if (!A_TMEM && !mbar_wait(&full[s], ph, abort_word, kErrWaitTma)) { ok = false; break; }
+        if (!A_TMEM && !mbar_wait(&full[s], ph, abort_word, kErrWaitTma)) break;
         __syncwarp();
         if (lane == 0) mbar_arrive(&prod[s]);
       }
     }
+  } else {
     // ------------------------------------------------------------------ epilogue
-    // Each group reads its half of the accumulator columns (group 0 all of them when BN < 64).
+    // Warp w drains TMEM lanes 32 (w % 4) .. + 31 (one output row per thread), chunk by chunk.
+    // With one accumulator (A in TMEM) eight warps each take half of the 256 columns and the
+    // next tile's MMAs wait for the drain (its loads and dequant proceed meanwhile); with two
+    // accumulators four warps drain all columns while the next tile's MMAs run in the other
+    // buffer.
+    const int e = warp - kEpiWarp0;
+    const int q = warp & 3;
     constexpr int kChunk = BN < 32 ? BN : 32;
-    const int c_begin = (BN < 64) ? 0 : grp * (BN / 2);
-    const int c_end = (BN < 64) ? (grp == 0 ? BN : 0) : c_begin + BN / 2;
-    if (c_begin < c_end && mbar_wait(accfull, 0u, abort_word, kErrWaitMma)) {
+    constexpr int kCols = A_TMEM ? BN / 2 : BN;   // columns this warp drains
+    const int c_base = A_TMEM ? (e >> 2) * (BN / 2) : 0;
+    const int tiles_m = (p.rows + kBM - 1) / kBM;
+    const int tiles_n = (p.cols + BN - 1) / BN;
+    const int64_t ntiles = (int64_t)tiles_m * tiles_n * p.splits;
+    int64_t tc = 0;
+    for (int64_t tt = blockIdx.x; tt < ntiles; tt += gridDim.x, ++tc) {
+      const TileInfo ti = tile_info<BN>(p, tiles_m, tiles_n, tt);
+      const int buf = (int)(tc % NB);
+      const uint32_t use = (uint32_t)(tc / NB) & 1u;
+      if (!mbar_wait(&accfull[buf], use, abort_word, kErrWaitMma)) break;
       tc_fence_after();
-      const int q = warp & 3;
-      const int row = row0 + 32 * q + lane;
+      const int row = ti.row0 + 32 * q + lane;
       const bool row_ok = row < p.rows;
+      const uint32_t taddr0 = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * C::kAccStride + c_base);
+      {
 #pragma unroll 1
-      for (int c0 = c_begin; c0 < c_end; c0 += kChunk) {
-        uint32_t r[32];
-        const uint32_t taddr = tmem_acc + ((uint32_t)(32 * q) << 16) + (uint32_t)c0;
-        if constexpr (kChunk == 32) tmem_ld_32x32b_x32(taddr, r);
-        else tmem_ld_32x32b_x16(taddr, r);
-        tmem_ld_wait();
-        if (!row_ok) continue;
-        if (p.epi == kEpiBf16T) {
-          uint16_t* out = reinterpret_cast<uint16_t*>(p.out);
+        for (int c0 = 0; c0 < kCols; c0 += kChunk) {
+          uint32_t r[32];
+          if constexpr (kChunk == 32) tmem_ld_32x32b_x32(taddr0 + (uint32_t)c0, r);
+          else tmem_ld_32x32b_x16(taddr0 + (uint32_t)c0, r);
+          tmem_ld_wait();
+          if (!row_ok) continue;
+          if (p.epi == kEpiBf16T) {
+            uint16_t* out = reinterpret_cast<uint16_t*>(p.out);
 #pragma unroll
-          for (int j = 0; j < kChunk; ++j) {
-            const int col = col0 + c0 + j;
-            if (col < p.cols) out[(int64_t)col * p.ld_out + row] = f32_to_bf16_bits(__uint_as_float(r[j]));
-          }
-        } else {
-          float* out = reinterpret_cast<float*>(p.out) + (int64_t)split * p.split_stride;
+            for (int j = 0; j < kChunk; ++j) {
+              const int col = ti.col0 + c_base + c0 + j;
+              if (col < p.cols) out[(int64_t)col * p.ld_out + row] = f32_to_bf16_bits(__uint_as_float(r[j]));
+            }
+          } else {
+            float* out = reinterpret_cast<float*>(p.out) + (int64_t)ti.split * p.split_stride;
 #pragma unroll
-          for (int j = 0; j < kChunk; ++j) {
-            const int col = col0 + c0 + j;
-            if (col < p.cols) out[(int64_t)col * p.ld_out + row] = __uint_as_float(r[j]);
+            for (int j = 0; j < kChunk; ++j) {
+              const int col = ti.col0 + c_base + c0 + j;
+              if (col < p.cols) out[(int64_t)col * p.ld_out + row] = __uint_as_float(r[j]);
+            }
           }
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&accempty[buf]);
       }
     }
-    tc_fence_before();
   }
 
+  tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_acc, C::kTmemCols);
+    tmem_dealloc(tmem_base, C::kTmemCols);
   }
 }
 
@@ -541,8 +685,11 @@ static cudaError_t launch_bn(const GemmParams& p, cudaStream_t st) {
   static std::atomic<uint64_t> configured{0};
   cudaError_t e = enable_smem_once(qlora_gemm_kernel<BN, GENERIC, A_TMEM>, C::kSmemBytes, configured);
   if (e != cudaSuccess) return e;
-  dim3 grid((p.rows + kBM - 1) / kBM, (p.cols + BN - 1) / BN, p.splits);
-  qlora_gemm_kernel<BN, GENERIC, A_TMEM><<<grid, kThreads, C::kSmemBytes, st>>>(p);
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t ntiles = (int64_t)((p.rows + kBM - 1) / kBM) * ((p.cols + BN - 1) / BN) * p.splits;
+  const int grid = (int)(ntiles < sms ? ntiles : sms);
+  qlora_gemm_kernel<BN, GENERIC, A_TMEM><<<grid, C::kThreads, C::kSmemBytes, st>>>(p);
   return cudaGetLastError();
 }
 
