@@ -330,6 +330,67 @@ __device__ __forceinline__ void tma_load_2d_hint(void* smem_dst, const CUtensorM
       : "memory");
 }
 
+// In-warp transpose of 8 x 8 bf16 values within each group of 8 lanes: on entry lane j holds
+// elements (j, 0..7) as four packed pairs x0..x3, on exit elements (0..7, j).  Three exchange
+// stages swap the off-diagonal blocks of 4, 2 and 1 elements with the lane at xor distance
+// 4, 2 and 1.
+__device__ __forceinline__ void transpose8x8_bf16(uint32_t& x0, uint32_t& x1, uint32_t& x2, uint32_t& x3, int lane) {
+  const bool b2 = lane & 4, b1 = lane & 2, b0 = lane & 1;
+  {
+    const uint32_t s0 = b2 ? x0 : x2, s1 = b2 ? x1 : x3;
+    const uint32_t r0 = __shfl_xor_sync(0xFFFFFFFFu, s0, 4), r1 = __shfl_xor_sync(0xFFFFFFFFu, s1, 4);
+    if (b2) { x0 = r0; x1 = r1; } else { x2 = r0; x3 = r1; }
+  }
+  {
+    const uint32_t s0 = b1 ? x0 : x1, s1 = b1 ? x2 : x3;
+    const uint32_t r0 = __shfl_xor_sync(0xFFFFFFFFu, s0, 2), r1 = __shfl_xor_sync(0xFFFFFFFFu, s1, 2);
+    if (b1) { x0 = r0; x2 = r1; } else { x1 = r0; x3 = r1; }
+  }
+  uint32_t* x[4] = {&x0, &x1, &x2, &x3};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t v = *x[k];
+    const uint32_t send = b0 ? (v & 0xFFFFu) : (v >> 16);
+    const uint32_t recv = __shfl_xor_sync(0xFFFFFFFFu, send, 1);
+    *x[k] = b0 ? ((v & 0xFFFF0000u) | recv) : ((v & 0xFFFFu) | (recv << 16));
+  }
+}
+
+// The MMA issuer's inner loop over `count` k-blocks of one stretch (one A layout).  The tensor
+// pipe queues only about one MMA ahead of the issuing thread, so the time this thread spends
+// between two k-blocks is pipe idle time: the ready barrier is polled inline (the bounded
+// wait only when the phase is not complete yet), ring positions and descriptors come from
+// incremental 32-bit counters, and the last k-block of a stretch is ragged only when
+// `k16_tail` < 4.  Returns false if a wait gave up.
+template <int BN, bool A_TMEM, bool A_MN, int S>
+__device__ __forceinline__ bool mma_run(int count, int k16_tail, uint64_t* ready, uint64_t* empty, uint32_t ready_err,
+                                        volatile uint32_t* abort_word, uint32_t smem_base, uint32_t tmem_base,
+                                        uint32_t tmem_acc, bool first, int& s, uint32_t& ph) {
+  using C = Cfg<BN, A_TMEM>;
+  for (int j = 0; j < count; ++j) {
+    if (!mbar_try_wait(&ready[s], ph))
+      if (!mbar_wait_thread(&ready[s], ph, abort_word, ready_err)) return false;
+    tc_fence_after();
+    const uint32_t a_addr = smem_base + (uint32_t)s * (uint32_t)C::kStageBytes;
+    const uint32_t b_addr = a_addr + (uint32_t)C::kABytes;
+    const uint32_t acc = (first && j == 0) ? 0u : 1u;
+    const int nk16 = (j == count - 1) ? k16_tail : 4;
+    if constexpr (A_TMEM) {
+      umma_kblock_ts<BN>(tmem_acc, tmem_base + kATmemCol0 + 32u * (uint32_t)s, b_addr, acc, nk16);
+    } else if (nk16 == 4) {
+      umma_kblock<BN, A_MN>(tmem_acc, a_addr, b_addr, acc);
+    } else {
+      umma_kblock_ragged<BN>(tmem_acc, a_addr, b_addr, acc, A_MN, nk16);
+    }
+    umma_commit(&empty[s]);
+    if (++s == S) {
+      s = 0;
+      ph ^= 1u;
+    }
+  }
+  return true;
+}
+
 template <int BN, bool GENERIC, bool A_TMEM>
 __global__ void __launch_bounds__(Cfg<BN, A_TMEM>::kThreads, 1) qlora_gemm_kernel(const __grid_constant__ GemmParams p) {
   using C = Cfg<BN, A_TMEM>;
@@ -472,31 +533,22 @@ __global__ void __launch_bounds__(Cfg<BN, A_TMEM>::kThreads, 1) qlora_gemm_kerne
         if (!mbar_wait_thread(&accempty[buf], use ^ 1u, abort_word, kErrWaitMma)) { ok = false; break; }
         tc_fence_after();
         const uint32_t tmem_acc = tmem_base + (uint32_t)(buf * C::kAccStride);
-        const bool first_split = ti.split == 0;
-        for (int it = 0; it < ti.n_iters; ++it) {
-          if (!mbar_wait_thread(&ready[s], ph, abort_word, ready_err)) { ok = false; break; }
-          tc_fence_after();
-          const IterPos ip = iter_pos(p, it, ti.kb_begin, ti.kb_end, first_split);
-          const GemmSeg& sg = p.seg[ip.seg];
+        const uint32_t smem_base = smem_u32(smem);
+        // segment 0 over this tile's K range, then (split 0) the adapter stretches
+        bool first = true;
+        for (int sgi = 0; sgi < p.nseg && ok; ++sgi) {
+          if (sgi > 0 && ti.split != 0) break;
+          const GemmSeg sg = p.seg[sgi];
+          const int count = sgi == 0 ? ti.kb_end - ti.kb_begin : sg.kblocks;
+          if (count <= 0) continue;
+          const bool ends = sgi > 0 || ti.kb_end == sg.kblocks;   // the stretch's last k-block is in this run
+          const int k16_tail = ends ? sg.k16_last : 4;
           const bool a_mn = (sg.a_src == kANf4MN || sg.a_src == kATmaMN);
-          const uint32_t a_addr = smem_u32(stage_a(s));
-          const uint32_t b_addr = smem_u32(stage_b(s));
-          const uint32_t acc = it > 0 ? 1u : 0u;
-          if constexpr (A_TMEM) {
-            (void)a_mn; (void)a_addr;
-            umma_kblock_ts<BN>(tmem_acc, tmem_base + kATmemCol0 + 32u * (uint32_t)s, b_addr, acc,
-                               ip.last ? sg.k16_last : 4);
-          } else if (!ip.last || sg.k16_last == 4) {
-            if (a_mn) umma_kblock<BN, true>(tmem_acc, a_addr, b_addr, acc);
-            else umma_kblock<BN, false>(tmem_acc, a_addr, b_addr, acc);
-          } else {
-            umma_kblock_ragged<BN>(tmem_acc, a_addr, b_addr, acc, a_mn, sg.k16_last);
-          }
-          umma_commit(&empty[s]);
-          if (++s == S) {
-            s = 0;
-            ph ^= 1u;
-          }
+          ok = a_mn ? mma_run<BN, A_TMEM, true, S>(count, k16_tail, ready, empty, ready_err, abort_word, smem_base,
+                                                    tmem_base, tmem_acc, first, s, ph)
+                    : mma_run<BN, A_TMEM, false, S>(count, k16_tail, ready, empty, ready_err, abort_word, smem_base,
+                                                     tmem_base, tmem_acc, first, s, ph);
+          first = false;
         }
         if (ok) umma_commit(&accfull[buf]);
       }
@@ -647,6 +699,27 @@ __global__ void __launch_bounds__(Cfg<BN, A_TMEM>::kThreads, 1) qlora_gemm_kerne
           if constexpr (kChunk == 32) tmem_ld_32x32b_x32(taddr0 + (uint32_t)c0, r);
           else tmem_ld_32x32b_x16(taddr0 + (uint32_t)c0, r);
           tmem_ld_wait();
+          if constexpr (kChunk == 32) {
+            if (p.epi == kEpiBf16T) {
+              // bf16 pairs, then an 8 x 8 transpose per group of 8 lanes: lane j of a group
+              // ends up with 8 consecutive output features of token j of each 8-token block,
+              // one 16-byte store instead of eight 2-byte ones
+              uint32_t w[16];
+#pragma unroll
+              for (int k = 0; k < 16; ++k) w[k] = pack_bf16x2(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1]));
+              const int fbase = ti.row0 + 32 * q + (lane & ~7);
+              uint16_t* out = reinterpret_cast<uint16_t*>(p.out);
+#pragma unroll
+              for (int b = 0; b < 4; ++b) {
+                uint32_t x0 = w[4 * b], x1 = w[4 * b + 1], x2 = w[4 * b + 2], x3 = w[4 * b + 3];
+                transpose8x8_bf16(x0, x1, x2, x3, lane);
+                const int col = ti.col0 + c_base + c0 + 8 * b + (lane & 7);
+                if (col < p.cols && fbase < p.rows)
+                  *reinterpret_cast<uint4*>(out + (int64_t)col * p.ld_out + fbase) = make_uint4(x0, x1, x2, x3);
+              }
+              continue;
+            }
+          }
           if (!row_ok) continue;
           if (p.epi == kEpiBf16T) {
             uint16_t* out = reinterpret_cast<uint16_t*>(p.out);
