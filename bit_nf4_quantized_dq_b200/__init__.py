@@ -13,14 +13,16 @@ from .binding import (  # noqa: F401
     lib,
     library_path,
     linear_plan,
+    merge_requantize,
     nf4_dequant,
     nf4_quantize_dq,
     qlora_linear_bwd,
     qlora_linear_fwd,
+    quantize,
     set_timing_events,
 )
 
 __all__ = [
-    "NF4Tensor", "QNF4Error", "check_device_error", "e4m3_encode", "lib", "library_path", "linear_plan", "set_timing_events",
-    "nf4_dequant", "nf4_quantize_dq", "qlora_linear_bwd", "qlora_linear_fwd",
+    "NF4Tensor", "QNF4Error", "check_device_error", "e4m3_encode", "lib", "library_path", "linear_plan", "merge_requantize", "set_timing_events",
+    "nf4_dequant", "nf4_quantize_dq", "qlora_linear_bwd", "qlora_linear_fwd", "quantize",
 ]

@@ -42,6 +42,20 @@ SIGNATURES = {
                                  c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_float,
                                  c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "nf4_e4m3_encode": (c_int, [c_void_p, c_int64, c_void_p, c_int, c_void_p]),
+    "qnf4_quantize_workspace_bytes_ex": (c_size_t, [c_int64, c_int]),
+    "qnf4_quantize_ex": (c_int, [c_void_p, c_int64, c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                 c_size_t, c_void_p]),
+    "qnf4_dequant_ex": (c_int, [c_void_p, c_int, c_int, c_void_p, c_void_p, c_void_p, c_int64, c_void_p, c_void_p]),
+    "qlora_linear_fwd_ex": (c_int, [c_void_p, c_int64, c_int64, c_int64, c_int, c_int, c_void_p, c_void_p,
+                                    c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_float, c_void_p, c_void_p,
+                                    c_void_p, c_size_t, c_void_p]),
+    "qlora_merge_workspace_bytes": (c_size_t, [c_int64, c_int64, c_int, c_int]),
+    "qlora_merge_requantize": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_int, c_int,
+                                       c_void_p, c_void_p, c_int, c_float, c_void_p, c_void_p, c_void_p, c_void_p,
+                                       c_void_p, c_void_p, c_size_t, c_void_p]),
+    "qlora_linear_bwd_ex": (c_int, [c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_int64, c_int, c_int,
+                                    c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_float,
+                                    c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "qnf4_set_timing_events": (c_int, [c_void_p, c_int]),
     "qlora_linear_plan": (c_int, [c_int64, c_int64, c_int64, c_int, ctypes.POINTER(c_int),
                                   ctypes.POINTER(c_int), ctypes.POINTER(c_int), ctypes.POINTER(c_int)]),
@@ -115,15 +129,33 @@ def check_device_error() -> int:
     return word.value
 
 
-class NF4Tensor:
-    """A quantized weight: codes, E4M3 scale codes, fp32 group constants, fp32 mean."""
+CODEBOOKS = {"nf4": 0, "fp4_e2m1": 1, "int4": 2}   # QNF4_CODEBOOK_* in include/qlora_nf4.h
 
-    def __init__(self, codes, scale_codes, c2, mean, shape):
+
+class NF4Tensor:
+    """A quantized weight: 4-bit codes and their block scales.
+
+    With double quantization (the default): E4M3 scale codes, fp32 group constants `c2` and
+    the fp32 mean.  Without it: `c2` holds one fp32 absmax per block and `scale_codes` and
+    `mean` are None.  `codebook` names the 16 levels ("nf4", "fp4_e2m1" or "int4")."""
+
+    def __init__(self, codes, scale_codes, c2, mean, shape, codebook: str = "nf4", double_quant: bool = True):
+        if codebook not in CODEBOOKS:
+            raise QNF4Error(f"unknown code book {codebook!r}")
         self.codes = codes
         self.scale_codes = scale_codes
         self.c2 = c2
         self.mean = mean
         self.shape = tuple(shape)
+        self.codebook = codebook
+        self.double_quant = bool(double_quant)
+
+    @property
+    def scales(self):
+        return self.c2
+
+    def _format(self):
+        return CODEBOOKS[self.codebook], 1 if self.double_quant else 0
 
     @property
     def numel(self) -> int:
@@ -133,7 +165,41 @@ class NF4Tensor:
         return n
 
     def nbytes(self) -> int:
-        return (self.codes.numel() + self.scale_codes.numel() + 4 * self.c2.numel() + 4 * self.mean.numel())
+        n = self.codes.numel() + 4 * self.c2.numel()
+        if self.double_quant:
+            n += self.scale_codes.numel() + 4 * self.mean.numel()
+        return n
+
+
+def quantize(W: torch.Tensor, codebook: str = "nf4", double_quant: bool = True,
+             workspace: Optional[torch.Tensor] = None) -> NF4Tensor:
+    """Blockwise 4-bit quantization of a bf16 weight with any of the code books, with or
+    without double quantization of the block scales."""
+    if codebook == "nf4" and double_quant:
+        return nf4_quantize_dq(W, workspace)
+    W = _bf16_bits(W)
+    _require_cuda(W)
+    numel = W.numel()
+    nb = (numel + 63) // 64
+    ng = (nb + 255) // 256
+    dev = W.device
+    codes = torch.empty(32 * nb, dtype=torch.uint8, device=dev)
+    if double_quant:
+        sc = torch.empty(nb, dtype=torch.uint8, device=dev)
+        scales = torch.empty(ng, dtype=torch.float32, device=dev)
+        mean = torch.empty(1, dtype=torch.float32, device=dev)
+    else:
+        sc, mean = None, None
+        scales = torch.empty(nb, dtype=torch.float32, device=dev)
+    out = NF4Tensor(codes, sc, scales, mean, W.shape, codebook, double_quant)
+    cb, dq = out._format()
+    L = lib()
+    need = L.qnf4_quantize_workspace_bytes_ex(numel, dq)
+    if workspace is None or workspace.numel() < need:
+        workspace = _ws(need, dev)
+    _check(L.qnf4_quantize_ex(_ptr(W), numel, cb, dq, _ptr(codes), _ptr(sc), _ptr(scales), _ptr(mean),
+                              _ptr(workspace), workspace.numel(), _stream()), "qnf4_quantize_ex")
+    return out
 
 
 def nf4_quantize_dq(W: torch.Tensor, workspace: Optional[torch.Tensor] = None) -> NF4Tensor:
@@ -200,8 +266,9 @@ def nf4_dequant(q: NF4Tensor, out: Optional[torch.Tensor] = None) -> torch.Tenso
     if out is None:
         out = torch.empty(q.shape, dtype=torch.bfloat16, device=q.codes.device)
     _require_cuda(out, q.codes)
-    _check(lib().nf4_dequant(_ptr(q.codes), _ptr(q.scale_codes), _ptr(q.c2), _ptr(q.mean), q.numel,
-                             _ptr(out), _stream()), "nf4_dequant")
+    cb, dq = q._format()
+    _check(lib().qnf4_dequant_ex(_ptr(q.codes), cb, dq, _ptr(q.scale_codes), _ptr(q.c2), _ptr(q.mean), q.numel,
+                                 _ptr(out), _stream()), "qnf4_dequant_ex")
     return out
 
 
@@ -220,9 +287,10 @@ def qlora_linear_fwd(x: torch.Tensor, q: NF4Tensor, A: torch.Tensor, B: torch.Te
     need = L.qlora_linear_fwd_workspace_bytes(M, K, N, r)
     if workspace is None or workspace.numel() < need:
         workspace = _ws(need, x.device)
-    _check(L.qlora_linear_fwd(_ptr(x), M, K, N, _ptr(q.codes), _ptr(q.scale_codes), _ptr(q.c2), _ptr(q.mean),
-                              _ptr(A), _ptr(B), r, float(s), _ptr(y), _ptr(t), _ptr(workspace),
-                              workspace.numel(), _stream()), "qlora_linear_fwd")
+    cb, dq = q._format()
+    _check(L.qlora_linear_fwd_ex(_ptr(x), M, K, N, cb, dq, _ptr(q.codes), _ptr(q.scale_codes), _ptr(q.c2),
+                                 _ptr(q.mean), _ptr(A), _ptr(B), r, float(s), _ptr(y), _ptr(t), _ptr(workspace),
+                                 workspace.numel(), _stream()), "qlora_linear_fwd")
     return y, t
 
 
@@ -241,10 +309,43 @@ def qlora_linear_bwd(dY: torch.Tensor, x: torch.Tensor, t_saved: torch.Tensor, q
     need = L.qlora_linear_bwd_workspace_bytes(M, K, N, r)
     if workspace is None or workspace.numel() < need:
         workspace = _ws(need, x.device)
-    _check(L.qlora_linear_bwd(_ptr(dY), _ptr(x), _ptr(t_saved), M, K, N, _ptr(q.codes), _ptr(q.scale_codes),
-                              _ptr(q.c2), _ptr(q.mean), _ptr(A), _ptr(B), r, float(s), _ptr(dX), _ptr(dA),
-                              _ptr(dB), _ptr(workspace), workspace.numel(), _stream()), "qlora_linear_bwd")
+    cb, dq = q._format()
+    _check(L.qlora_linear_bwd_ex(_ptr(dY), _ptr(x), _ptr(t_saved), M, K, N, cb, dq, _ptr(q.codes),
+                                 _ptr(q.scale_codes), _ptr(q.c2), _ptr(q.mean), _ptr(A), _ptr(B), r, float(s),
+                                 _ptr(dX), _ptr(dA), _ptr(dB), _ptr(workspace), workspace.numel(), _stream()),
+           "qlora_linear_bwd")
     return dX, dA, dB
+
+
+def merge_requantize(q: NF4Tensor, A: torch.Tensor, B: torch.Tensor, s: float, return_merged: bool = False):
+    """Fold the adapters into the base and quantize the result again in the same format:
+    W'' = bf16(W' + s B A), then quantized.  Returns the new NF4Tensor (and W'' as a bf16
+    tensor when `return_merged`)."""
+    _require_cuda(A, B, q.codes)
+    N, K = q.shape
+    r = A.shape[0]
+    if tuple(A.shape) != (r, K) or tuple(B.shape) != (N, r):
+        raise QNF4Error("shape mismatch between W, A and B")
+    dev = q.codes.device
+    nb = (N * K + 63) // 64
+    ng = (nb + 255) // 256
+    codes = torch.empty(32 * nb, dtype=torch.uint8, device=dev)
+    if q.double_quant:
+        sc = torch.empty(nb, dtype=torch.uint8, device=dev)
+        scales = torch.empty(ng, dtype=torch.float32, device=dev)
+        mean = torch.empty(1, dtype=torch.float32, device=dev)
+    else:
+        sc, mean = None, None
+        scales = torch.empty(nb, dtype=torch.float32, device=dev)
+    out = NF4Tensor(codes, sc, scales, mean, (N, K), q.codebook, q.double_quant)
+    merged = torch.empty((N, K), dtype=torch.bfloat16, device=dev) if return_merged else None
+    cb, dq = q._format()
+    L = lib()
+    ws = _ws(L.qlora_merge_workspace_bytes(N, K, dq, 1 if merged is not None else 0), dev)
+    _check(L.qlora_merge_requantize(_ptr(q.codes), _ptr(q.scale_codes), _ptr(q.c2), _ptr(q.mean), N, K, cb, dq,
+                                    _ptr(A), _ptr(B), r, float(s), _ptr(codes), _ptr(sc), _ptr(scales), _ptr(mean),
+                                    _ptr(merged), _ptr(ws), ws.numel(), _stream()), "qlora_merge_requantize")
+    return (out, merged) if return_merged else out
 
 
 def set_timing_events(events) -> None:

@@ -30,8 +30,8 @@ struct __align__(8) BucketEntry {
 
 // Thread b < 33 computes bucket b once and fills its 32 per-lane copies (one copy per lane
 // keeps the lookups of a warp free of bank conflicts).
-__device__ __forceinline__ void build_bucket_table(BucketEntry (*tab)[32]) {
-  constexpr float q[16] = QNF4_LEVELS;
+__device__ __forceinline__ void build_bucket_table(BucketEntry (*tab)[32], const Codebook& cb) {
+  const float* q = cb.q;
   const int b = threadIdx.x;
   if (b >= 33) return;
   // bucket b holds the fp32 n with round(16 n + 16) == b
@@ -141,6 +141,7 @@ constexpr int kQSmemBytes = kQStages * kQStageBytes + 1024;
 
 struct QuantParams {
   CUtensorMap w_map;          // W as [nb_full][64] bf16, box 64 x 256, 128-byte swizzle
+  Codebook cb;
   const uint16_t* W;
   int64_t numel, nb, nb_full, ng;
   uint32_t* codes32;
@@ -164,7 +165,7 @@ __global__ void __launch_bounds__(kQThreads, 2) nf4_quant_stream_kernel(const __
     abort_flag = 0u;
     mbar_fence_init();
   }
-  build_bucket_table(tab);
+  build_bucket_table(tab, p.cb);
   __syncthreads();
   volatile uint32_t* abort_word = &abort_flag;
   const int64_t n_local = p.ng > blockIdx.x ? (p.ng - 1 - blockIdx.x) / gridDim.x + 1 : 0;
@@ -266,7 +267,7 @@ __global__ void __launch_bounds__(kQThreads, 2) nf4_quant_stream_kernel(const __
       // buffers, so thread 0 reads this group's while the warps fill the other one
       asm volatile("bar.sync 1, %0;" ::"r"(32 * kQGroupWarps) : "memory");
       if (*abort_word) break;
-      if (t == 0) {
+      if (t == 0 && p.gsum != nullptr) {   // no group sums without double quantization
         const double* w = warp_sum[parity];
         const double q0 = ((w[0] + w[1]) + (w[2] + w[3])) + ((w[4] + w[5]) + (w[6] + w[7]));
         const double q1 = ((w[8] + w[9]) + (w[10] + w[11])) + ((w[12] + w[13]) + (w[14] + w[15]));
@@ -409,7 +410,8 @@ __global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint8_t* __restr
                                                           const uint8_t* __restrict__ scale_codes,
                                                           const float* __restrict__ c2,
                                                           const float* __restrict__ mean_p, int64_t numel,
-                                                          int64_t nb, uint16_t* __restrict__ out) {
+                                                          int64_t nb, uint16_t* __restrict__ out, const Codebook cb,
+                                                          int scale_fp32) {
   __shared__ uint4 stage[8][32 * 8];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t b0 = (int64_t)blockIdx.x * blockDim.x + warp * 32;   // first block of this warp
@@ -419,8 +421,9 @@ __global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint8_t* __restr
   uint32_t w[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   Nf4Lut L{};
   if (b < nb) {
-    const float scale = dq_block_scale(__ldg(scale_codes + b), __ldg(c2 + (b >> 8)), __ldg(mean_p));
-    nf4_lut_build(scale, L);
+    // scale_fp32: c2 holds the fp32 absmax of every block (single-level quantization)
+    const float scale = scale_fp32 ? __ldg(c2 + b) : dq_block_scale(__ldg(scale_codes + b), __ldg(c2 + (b >> 8)), __ldg(mean_p));
+    nf4_lut_build(scale, L, cb);
     const uint4* src = reinterpret_cast<const uint4*>(codes + b * 32);
     const uint4 c0 = __ldg(src), c1 = __ldg(src + 1);
     w[0] = c0.x; w[1] = c0.y; w[2] = c0.z; w[3] = c0.w;
@@ -477,9 +480,9 @@ static int grid_for(int64_t threads, int per_block, int cap) {
   return (int)g;
 }
 
-cudaError_t launch_quantize(const CUtensorMap* w_map, const uint16_t* W, int64_t numel, uint8_t* codes,
-                            uint8_t* scale_codes, float* c2, float* mean, float* absmax_ws, double* gsum_ws,
-                            cudaStream_t st, int sw_encode) {
+cudaError_t launch_quantize(const CUtensorMap* w_map, const uint16_t* W, int64_t numel, const Codebook& cb,
+                            uint8_t* codes, uint8_t* scale_codes, float* c2, float* mean, float* absmax_ws,
+                            double* gsum_ws, cudaStream_t st, int sw_encode) {
   const int64_t nb = (numel + kB1 - 1) / kB1;
   const int64_t ng = (nb + kB2 - 1) / kB2;
   if (ng > (int64_t)kMaxMeanChunks * 2048) return cudaErrorInvalidValue;
@@ -492,6 +495,7 @@ cudaError_t launch_quantize(const CUtensorMap* w_map, const uint16_t* W, int64_t
   QuantParams qp;
   memset(&qp, 0, sizeof(qp));
   if (w_map) qp.w_map = *w_map;
+  qp.cb = cb;
   qp.W = W;
   qp.numel = numel;
   qp.nb = nb;
@@ -503,6 +507,7 @@ cudaError_t launch_quantize(const CUtensorMap* w_map, const uint16_t* W, int64_t
   nf4_quant_stream_kernel<<<grid_for(ng, 1, 2 * sms), kQThreads, kQSmemBytes, st>>>(qp);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  if (!gsum_ws) return cudaSuccess;   // single-level quantization: the absmax values are the scales
   // The double-quantization kernel may launch while the quantize grid drains (programmatic
   // dependent launch); it waits for that grid's results before reading them.
   cudaLaunchConfig_t cfg = {};
@@ -528,9 +533,10 @@ cudaError_t launch_quantize(const CUtensorMap* w_map, const uint16_t* W, int64_t
 }
 
 cudaError_t launch_dequant(const uint8_t* codes, const uint8_t* scale_codes, const float* c2, const float* mean,
-                           int64_t numel, uint16_t* out, cudaStream_t st) {
+                           int64_t numel, uint16_t* out, const Codebook& cb, int scale_fp32, cudaStream_t st) {
   const int64_t nb = (numel + kB1 - 1) / kB1;
-  nf4_dequant_kernel<<<grid_for(nb, 256, 1 << 30), 256, 0, st>>>(codes, scale_codes, c2, mean, numel, nb, out);
+  nf4_dequant_kernel<<<grid_for(nb, 256, 1 << 30), 256, 0, st>>>(codes, scale_codes, c2, mean, numel, nb, out, cb,
+                                                                  scale_fp32);
   return cudaGetLastError();
 }
 

@@ -144,29 +144,29 @@ __device__ __forceinline__ UnitGeom unit_geom(int a_src, int t, int row0, int64_
   return u;
 }
 
-// Raw per-unit scale data, fetched one iteration ahead of its use.
+// Per-unit block scales, fetched (and formed) one iteration ahead of their use.
 struct UnitScale {
-  uint32_t e0, e1;   // scale codes of the unit's block and (generic path) of the next block
-  float c20, c21;    // their group constants
+  float s0, s1;      // scale of the unit's block and (generic path) of the next block
   int32_t split;     // words before the block boundary (8 = one block), generic path only
   int32_t valid;     // valid 8-code words (0 = unit outside the weight)
 };
 
+__device__ __forceinline__ float block_scale_of(const GemmParams& p, int64_t blk, float mean) {
+  if (p.scale_fp32) return __ldg(p.c2 + blk);
+  return dq_block_scale(__ldg(p.scale_codes + blk), __ldg(p.c2 + (blk >> 8)), mean);
+}
+
 template <bool GENERIC>
-__device__ __forceinline__ UnitScale fetch_scale(const GemmParams& p, const UnitGeom& u, int64_t nb) {
-  UnitScale r{0u, 0u, 0.0f, 0.0f, 8, 0};
+__device__ __forceinline__ UnitScale fetch_scale(const GemmParams& p, const UnitGeom& u, int64_t nb, float mean) {
+  UnitScale r{0.0f, 0.0f, 8, 0};
   if (u.n >= p.nw || u.kcol >= p.kw) return r;
   const int64_t f0 = u.n * p.kw + u.kcol;
   const int64_t blk = f0 >> 6;
-  r.e0 = __ldg(p.scale_codes + blk);
-  r.c20 = __ldg(p.c2 + (blk >> 8));
+  r.s0 = block_scale_of(p, blk, mean);
   r.valid = 8;
   if constexpr (GENERIC) {
     r.split = (int32_t)((64 - (f0 & 63)) >> 3);
-    if (r.split < 8 && blk + 1 < nb) {
-      r.e1 = __ldg(p.scale_codes + blk + 1);
-      r.c21 = __ldg(p.c2 + ((blk + 1) >> 8));
-    }
+    if (r.split < 8 && blk + 1 < nb) r.s1 = block_scale_of(p, blk + 1, mean);
     const int64_t vw = (p.kw - u.kcol) >> 3;
     r.valid = (int32_t)(vw < 8 ? vw : 8);
   }
@@ -564,8 +564,9 @@ __global__ void __launch_bounds__(Cfg<BN, A_TMEM>::kThreads, 1) qlora_gemm_kerne
     const int grp = (warp - 2) >> 2;          // 0: warps 2-5, 1: warps 6-9
     const int t = 32 * (warp & 3) + lane;       // tile row t = TMEM lane t (warp w reaches lanes 32 (w % 4) ..)
     if (p.has_nf4) {
-      const float mean = __ldg(p.mean);
+      const float mean = p.scale_fp32 ? 0.0f : __ldg(p.mean);
       const int64_t nb = (p.nw * p.kw + kB1 - 1) / kB1;
+      const Codebook& cb = p.cb;
       auto geom = [&](const KIter<BN, S>& q, bool& nf4, UnitGeom& u) {
         const IterPos ip = iter_pos(p, q.it, q.ti.kb_begin, q.ti.kb_end, q.ti.split == 0);
         const GemmSeg& sg = p.seg[ip.seg];
@@ -580,7 +581,7 @@ __global__ void __launch_bounds__(Cfg<BN, A_TMEM>::kThreads, 1) qlora_gemm_kerne
       UnitScale sc_next{};
       if (!nxt.done) {
         geom(nxt, nf4_next, u_next);
-        if (nf4_next) sc_next = fetch_scale<GENERIC>(p, u_next, nb);
+        if (nf4_next) sc_next = fetch_scale<GENERIC>(p, u_next, nb, mean);
       }
       for (; !cur.done; cur.advance(p, 2)) {
         const int s = cur.stage;
@@ -591,14 +592,14 @@ __global__ void __launch_bounds__(Cfg<BN, A_TMEM>::kThreads, 1) qlora_gemm_kerne
         nxt.advance(p, 2);                    // prefetch the next k-block's scales
         if (!nxt.done) {
           geom(nxt, nf4_next, u_next);
-          if (nf4_next) sc_next = fetch_scale<GENERIC>(p, u_next, nb);
+          if (nf4_next) sc_next = fetch_scale<GENERIC>(p, u_next, nb, mean);
         }
         Nf4Lut L0, L1;
         uint32_t words[8];
         if (nf4) {
-          nf4_lut_build(sc.valid ? dq_block_scale(sc.e0, sc.c20, mean) : 0.0f, L0);
+          nf4_lut_build(sc.valid ? sc.s0 : 0.0f, L0, cb);
           if constexpr (GENERIC) {
-            if (sc.split < 8) nf4_lut_build(dq_block_scale(sc.e1, sc.c21, mean), L1);
+            if (sc.split < 8) nf4_lut_build(sc.s1, L1, cb);
             const uint32_t* src = reinterpret_cast<const uint32_t*>(p.codes + ((u.n * p.kw + u.kcol) >> 1));
 #pragma unroll
             for (int j = 0; j < 8; ++j) words[j] = (j < sc.valid) ? __ldg(src + j) : 0u;

@@ -5,6 +5,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include "codebook.h"
+
 namespace qnf4 {
 
 // Source of the A operand (the 128-row UMMA "M" side) for one stretch of the K loop.
@@ -48,12 +50,16 @@ struct GemmParams {
   int32_t a_tmem;
   const uint16_t* a_glob;
   int64_t a_glob_ld, a_glob_rows, a_glob_cols;
-  // NF4 operand: codes / scale codes / group constants / mean of W [nw][kw]
+  // 4-bit operand: codes / scale codes / group constants / mean of W [nw][kw], its 16 levels,
+  // and the scale format (scale_fp32 = 1: c2 holds one fp32 scale per block of 64, the
+  // single-level format without double quantization; scale_codes and mean are unused)
   const uint8_t* codes;
   const uint8_t* scale_codes;
   const float* c2;
   const float* mean;
   int64_t nw, kw;
+  Codebook cb;
+  int32_t scale_fp32;
   // epilogue
   int32_t epi;
   float alpha;

@@ -11,6 +11,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "codebook.h"
 
 namespace qnf4 {
 
@@ -68,18 +69,17 @@ __device__ __forceinline__ float dq_block_scale(uint32_t scale_code, float c2, f
 
 // ---------------------------------------------------------------------------------------
 // Per-block bf16 table: entry j = bf16(fp32(level_j * scale)), split into low and high
-// bytes so that 4 entries are selected by one byte permute.
+// bytes so that 4 entries are selected by one byte permute.  The default code book is NF4.
 // ---------------------------------------------------------------------------------------
 struct Nf4Lut {
   uint32_t lo[4];   // low bytes of entries 4k..4k+3
   uint32_t hi[4];   // high bytes of entries 4k..4k+3
 };
 
-__device__ __forceinline__ void nf4_lut_build(float scale, Nf4Lut& L) {
-  constexpr float q[16] = QNF4_LEVELS;
+__device__ __forceinline__ void nf4_lut_build(float scale, Nf4Lut& L, const Codebook& cb) {
   uint32_t P[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) P[i] = pack_bf16x2(__fmul_rn(q[2 * i], scale), __fmul_rn(q[2 * i + 1], scale));
+  for (int i = 0; i < 8; ++i) P[i] = pack_bf16x2(__fmul_rn(cb.q[2 * i], scale), __fmul_rn(cb.q[2 * i + 1], scale));
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     L.lo[k] = prmt(P[2 * k], P[2 * k + 1], 0x6420u);

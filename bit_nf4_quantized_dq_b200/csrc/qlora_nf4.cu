@@ -2,6 +2,7 @@
 // (argument checks, workspace layout, TMA tensor maps, kernel sequencing).
 #include <cstdarg>
 #include <cstdio>
+#include <cmath>
 #include <algorithm>
 #include <cstring>
 #include <mutex>
@@ -11,6 +12,7 @@
 #include "codec.cuh"
 #include "gemm.cuh"
 #include "lowrank.cuh"
+#include "merge.cuh"
 
 namespace {
 
@@ -279,16 +281,72 @@ int b_box_rows(int bn) { return bn; }
 
 cudaError_t launch_fused(const qnf4::GemmParams& gp, int bn, cudaStream_t st) { return qnf4::launch_gemm(gp, bn, st); }
 
-int nf4_operand(qnf4::GemmParams& gp, const uint8_t* codes, const uint8_t* scale_codes, const float* c2,
-                const float* mean, int64_t N, int64_t K) {
+// ------------------------------------------------------------------------ code books
+// NF4: the 8-decimal levels of the code book table, each the nearest fp32 (the compiler rounds
+// the literals).  FP4 E2M1: its 16 values 0, 0.5, 1, 1.5, 2, 3, 4, 6 (both signs, two zeros)
+// over 6, sorted.  INT4: 16 levels equally spaced over [-1, 1], -1 + 2 i / 15.  The quotients
+// are formed in double and rounded once to float; none of them lies near a float rounding
+// midpoint (their binary expansions repeat), so that is the nearest float.
+int get_codebook(int id, qnf4::Codebook* cb) {
+  static const float nf4[16] = QNF4_LEVELS;
+  switch (id) {
+    case QNF4_CODEBOOK_NF4:
+      for (int j = 0; j < 16; ++j) cb->q[j] = nf4[j];
+      break;
+    case QNF4_CODEBOOK_FP4_E2M1: {
+      static const double mags[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+      for (int j = 0; j < 8; ++j) {
+        cb->q[7 - j] = -(float)(mags[j] / 6.0);   // -0 at index 7
+        cb->q[8 + j] = (float)(mags[j] / 6.0);
+      }
+      break;
+    }
+    case QNF4_CODEBOOK_INT4:
+      for (int j = 0; j < 16; ++j) cb->q[j] = (float)((double)(2 * j - 15) / 15.0);
+      break;
+    default:
+      return fail(QNF4_ERR_INVALID, "unknown code book %d", id);
+  }
+  // The quantizer finds the nearest level through 33 buckets of width 1/16 over [-1, 1] and
+  // one threshold compare per bucket: every bucket may hold at most one threshold (the largest
+  // float not above a midpoint between neighbouring levels).
+  if (cb->q[0] != -1.0f || cb->q[15] != 1.0f) return fail(QNF4_ERR_INVALID, "code book must span [-1, 1]");
+  int count[33] = {0};
+  for (int j = 0; j < 15; ++j) {
+    if (!(cb->q[j] <= cb->q[j + 1])) return fail(QNF4_ERR_INVALID, "code book levels must not decrease");
+    const double m = 0.5 * ((double)cb->q[j] + (double)cb->q[j + 1]);
+    float th = (float)m;
+    if ((double)th > m) th = std::nextafter(th, -2.0f);
+    for (int b = 0; b < 33; ++b)
+      if ((double)th >= (b - 16.5) / 16.0 && (double)th < (b - 15.5) / 16.0) ++count[b];
+  }
+  for (int b = 0; b < 33; ++b)
+    if (count[b] > 1) return fail(QNF4_ERR_UNSUPPORTED, "code book: two midpoints share a quantizer bucket");
+  return QNF4_OK;
+}
+
+int nf4_operand(qnf4::GemmParams& gp, const qnf4::Codebook& cb, int double_quant, const uint8_t* codes,
+                const uint8_t* scale_codes, const float* scales, const float* mean, int64_t N, int64_t K) {
   gp.has_nf4 = 1;
   gp.nf4_generic = (K % 64 != 0) ? 1 : 0;
   gp.codes = codes;
   gp.scale_codes = scale_codes;
-  gp.c2 = c2;
+  gp.c2 = scales;
   gp.mean = mean;
   gp.nw = N;
   gp.kw = K;
+  gp.cb = cb;
+  gp.scale_fp32 = double_quant ? 0 : 1;
+  return QNF4_OK;
+}
+
+// Checks of the stored-format pointers: with double quantization scale codes, group constants
+// and the mean; without it, one fp32 scale per block (scale_codes and mean unused).
+int check_format(int double_quant, const uint8_t* codes, const uint8_t* scale_codes, const float* scales,
+                 const float* mean) {
+  if (double_quant != 0 && double_quant != 1) return fail(QNF4_ERR_INVALID, "double_quant must be 0 or 1");
+  if (!codes || !scales || (double_quant && (!scale_codes || !mean))) return fail(QNF4_ERR_INVALID, "NULL pointer");
+  if (!aligned(codes, 16)) return fail(QNF4_ERR_UNSUPPORTED, "codes need 16 B alignment");
   return QNF4_OK;
 }
 
@@ -382,47 +440,87 @@ int qnf4_device_error(void* stream, uint32_t* word) {
   return QNF4_OK;
 }
 
-size_t nf4_quantize_workspace_bytes(int64_t numel) {
+size_t nf4_quantize_workspace_bytes(int64_t numel) { return qnf4_quantize_workspace_bytes_ex(numel, 1); }
+
+size_t qnf4_quantize_workspace_bytes_ex(int64_t numel, int double_quant) {
   if (numel <= 0) return 0;
   const int64_t nb = (numel + 63) / 64, ng = (nb + 255) / 256;
+  if (!double_quant) return 256;   // the absmax values are the outputs; nothing else is needed
   return align_up((size_t)nb * 4, 256) + (size_t)ng * 8;
 }
 
-int nf4_quantize_dq(const uint16_t* W, int64_t numel, uint8_t* codes, uint8_t* scale_codes, float* c2, float* mean,
-                    void* workspace, size_t workspace_bytes, void* stream) {
-  g_last_error.clear();
-  if (!W || !codes || !scale_codes || !c2 || !mean || !workspace) return fail(QNF4_ERR_INVALID, "NULL pointer");
-  if (numel <= 0) return fail(QNF4_ERR_INVALID, "numel must be positive");
-  if (numel > (1ll << 35)) return fail(QNF4_ERR_UNSUPPORTED, "numel above 2^35");
-  if (!aligned(W, 16) || !aligned(codes, 16) || !aligned(scale_codes, 8) || !aligned(workspace, 256))
-    return fail(QNF4_ERR_UNSUPPORTED, "alignment: W and codes 16 B, scale_codes 8 B, workspace 256 B");
-  if (workspace_bytes < nf4_quantize_workspace_bytes(numel))
-    return fail(QNF4_ERR_WORKSPACE, "workspace needs %zu bytes", nf4_quantize_workspace_bytes(numel));
-  if (int rc = check_arch()) return rc;
-  const int64_t nb = (numel + 63) / 64;
-  float* absmax = static_cast<float*>(workspace);
-  double* gsum = reinterpret_cast<double*>(static_cast<char*>(workspace) + align_up((size_t)nb * 4, 256));
+}  // extern "C"
+
+namespace {
+
+// Quantize into caller buffers; absmax / gsum are the scratch of double quantization (unused
+// without it: the block absmax values go straight to `scales`).
+int quantize_impl(const uint16_t* W, int64_t numel, int codebook, int double_quant, uint8_t* codes,
+                  uint8_t* scale_codes, float* scales, float* mean, float* absmax, double* gsum, cudaStream_t st) {
+  qnf4::Codebook cb;
+  if (int rc = get_codebook(codebook, &cb)) return rc;
   CUtensorMap wmap;
   const bool has_map = numel >= 64;
   if (has_map)
     if (int rc = make_map(&wmap, W, true, 64, (uint64_t)(numel / 64), 128, 64, 256)) return rc;
-  cudaError_t e = qnf4::launch_quantize(has_map ? &wmap : nullptr, W, numel, codes, scale_codes, c2, mean, absmax, gsum,
-                                        static_cast<cudaStream_t>(stream), 0);
+  cudaError_t e = double_quant
+                      ? qnf4::launch_quantize(has_map ? &wmap : nullptr, W, numel, cb, codes, scale_codes, scales, mean,
+                                              absmax, gsum, st, 0)
+                      : qnf4::launch_quantize(has_map ? &wmap : nullptr, W, numel, cb, codes, nullptr, nullptr,
+                                              nullptr, scales, nullptr, st, 0);
   if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
   return QNF4_OK;
+}
+
+int check_quantize_args(const uint16_t* W, int64_t numel, int double_quant, uint8_t* codes, uint8_t* scale_codes,
+                        float* scales, float* mean) {
+  if (!W) return fail(QNF4_ERR_INVALID, "NULL pointer");
+  if (int rc = check_format(double_quant, codes, scale_codes, scales, mean)) return rc;
+  if (numel <= 0) return fail(QNF4_ERR_INVALID, "numel must be positive");
+  if (numel > (1ll << 35)) return fail(QNF4_ERR_UNSUPPORTED, "numel above 2^35");
+  if (!aligned(W, 16) || (double_quant && !aligned(scale_codes, 8)))
+    return fail(QNF4_ERR_UNSUPPORTED, "alignment: W and codes 16 B, scale_codes 8 B");
+  return QNF4_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int qnf4_quantize_ex(const uint16_t* W, int64_t numel, int codebook, int double_quant, uint8_t* codes,
+                     uint8_t* scale_codes, float* scales, float* mean, void* workspace, size_t workspace_bytes,
+                     void* stream) {
+  g_last_error.clear();
+  if (int rc = check_quantize_args(W, numel, double_quant, codes, scale_codes, scales, mean)) return rc;
+  if (double_quant) {
+    if (!workspace) return fail(QNF4_ERR_INVALID, "NULL pointer");
+    if (!aligned(workspace, 256)) return fail(QNF4_ERR_UNSUPPORTED, "workspace needs 256-byte alignment");
+    const size_t need = qnf4_quantize_workspace_bytes_ex(numel, 1);
+    if (workspace_bytes < need) return fail(QNF4_ERR_WORKSPACE, "workspace needs %zu bytes", need);
+  }
+  if (int rc = check_arch()) return rc;
+  const int64_t nb = (numel + 63) / 64;
+  float* absmax = double_quant ? static_cast<float*>(workspace) : nullptr;
+  double* gsum = double_quant ? reinterpret_cast<double*>(static_cast<char*>(workspace) + align_up((size_t)nb * 4, 256))
+                              : nullptr;
+  return quantize_impl(W, numel, codebook, double_quant, codes, scale_codes, scales, mean, absmax, gsum,
+                       static_cast<cudaStream_t>(stream));
+}
+
+int nf4_quantize_dq(const uint16_t* W, int64_t numel, uint8_t* codes, uint8_t* scale_codes, float* c2, float* mean,
+                    void* workspace, size_t workspace_bytes, void* stream) {
+  return qnf4_quantize_ex(W, numel, QNF4_CODEBOOK_NF4, 1, codes, scale_codes, c2, mean, workspace, workspace_bytes,
+                          stream);
 }
 
 int nf4_quantize_dq_noalloc(const uint16_t* W, int64_t numel, uint8_t* codes, uint8_t* scale_codes, float* c2,
                             float* mean, void* stream) {
   g_last_error.clear();
-  if (!W || !codes || !scale_codes || !c2 || !mean) return fail(QNF4_ERR_INVALID, "NULL pointer");
-  if (numel <= 0) return fail(QNF4_ERR_INVALID, "numel must be positive");
   if (numel > QNF4_NOALLOC_MAX_NUMEL)
     return fail(QNF4_ERR_UNSUPPORTED,
                 "numel %lld is above the static scratch limit of %lld weights; use nf4_quantize_dq with a workspace",
                 (long long)numel, (long long)QNF4_NOALLOC_MAX_NUMEL);
-  if (!aligned(W, 16) || !aligned(codes, 16) || !aligned(scale_codes, 8))
-    return fail(QNF4_ERR_UNSUPPORTED, "alignment: W and codes 16 B, scale_codes 8 B");
+  if (int rc = check_quantize_args(W, numel, 1, codes, scale_codes, c2, mean)) return rc;
   if (int rc = check_arch()) return rc;
   void* scratch = nullptr;
   if (int rc = noalloc_scratch(&scratch)) return rc;
@@ -430,26 +528,29 @@ int nf4_quantize_dq_noalloc(const uint16_t* W, int64_t numel, uint8_t* codes, ui
   const int64_t nb = (numel + 63) / 64;
   float* absmax = static_cast<float*>(scratch);
   double* gsum = reinterpret_cast<double*>(static_cast<char*>(scratch) + align_up((size_t)nb * 4, 256));
-  CUtensorMap wmap;
-  const bool has_map = numel >= 64;
-  if (has_map)
-    if (int rc = make_map(&wmap, W, true, 64, (uint64_t)(numel / 64), 128, 64, 256)) return rc;
-  cudaError_t e = qnf4::launch_quantize(has_map ? &wmap : nullptr, W, numel, codes, scale_codes, c2, mean, absmax, gsum,
-                                        static_cast<cudaStream_t>(stream), 0);
-  if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
+  return quantize_impl(W, numel, QNF4_CODEBOOK_NF4, 1, codes, scale_codes, c2, mean, absmax, gsum,
+                       static_cast<cudaStream_t>(stream));
+}
+
+int qnf4_dequant_ex(const uint8_t* codes, int codebook, int double_quant, const uint8_t* scale_codes,
+                    const float* scales, const float* mean, int64_t numel, uint16_t* W_out, void* stream) {
+  g_last_error.clear();
+  if (!W_out) return fail(QNF4_ERR_INVALID, "NULL pointer");
+  if (int rc = check_format(double_quant, codes, scale_codes, scales, mean)) return rc;
+  if (numel <= 0) return fail(QNF4_ERR_INVALID, "numel must be positive");
+  if (!aligned(W_out, 16)) return fail(QNF4_ERR_UNSUPPORTED, "codes and W_out need 16 B");
+  qnf4::Codebook cb;
+  if (int rc = get_codebook(codebook, &cb)) return rc;
+  if (int rc = check_arch()) return rc;
+  cudaError_t e = qnf4::launch_dequant(codes, scale_codes, scales, mean, numel, W_out, cb, double_quant ? 0 : 1,
+                                       static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "dequant launch");
   return QNF4_OK;
 }
 
 int nf4_dequant(const uint8_t* codes, const uint8_t* scale_codes, const float* c2, const float* mean,
                 int64_t numel, uint16_t* W_out, void* stream) {
-  g_last_error.clear();
-  if (!codes || !scale_codes || !c2 || !mean || !W_out) return fail(QNF4_ERR_INVALID, "NULL pointer");
-  if (numel <= 0) return fail(QNF4_ERR_INVALID, "numel must be positive");
-  if (!aligned(codes, 16) || !aligned(W_out, 16)) return fail(QNF4_ERR_UNSUPPORTED, "codes and W_out need 16 B");
-  if (int rc = check_arch()) return rc;
-  cudaError_t e = qnf4::launch_dequant(codes, scale_codes, c2, mean, numel, W_out, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "dequant launch");
-  return QNF4_OK;
+  return qnf4_dequant_ex(codes, QNF4_CODEBOOK_NF4, 1, scale_codes, c2, mean, numel, W_out, stream);
 }
 
 int nf4_e4m3_encode(const float* v, int64_t n, uint8_t* out, int mode, void* stream) {
@@ -461,6 +562,63 @@ int nf4_e4m3_encode(const float* v, int64_t n, uint8_t* out, int mode, void* str
   cudaError_t e = qnf4::launch_e4m3_encode(v, n, out, mode, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "e4m3 launch");
   return QNF4_OK;
+}
+
+size_t qlora_merge_workspace_bytes(int64_t N, int64_t K, int double_quant, int merged_out_given) {
+  if (N <= 0 || K <= 0) return 0;
+  const size_t merged = merged_out_given ? 0 : align_up((size_t)N * (size_t)K * 2, 256);
+  return merged + qnf4_quantize_workspace_bytes_ex(N * K, double_quant);
+}
+
+int qlora_merge_requantize(const uint8_t* codes, const uint8_t* scale_codes, const float* scales, const float* mean,
+                           int64_t N, int64_t K, int codebook, int double_quant, const uint16_t* A, const uint16_t* B,
+                           int r, float s, uint8_t* codes_out, uint8_t* scale_codes_out, float* scales_out,
+                           float* mean_out, uint16_t* merged_out, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+  g_last_error.clear();
+  if (!A || !B || !workspace) return fail(QNF4_ERR_INVALID, "NULL pointer");
+  if (int rc = check_format(double_quant, codes, scale_codes, scales, mean)) return rc;
+  if (int rc = check_format(double_quant, codes_out, scale_codes_out, scales_out, mean_out)) return rc;
+  if (N <= 0 || K <= 0 || r <= 0) return fail(QNF4_ERR_INVALID, "sizes must be positive");
+  if (K % 8 || r > 1024) return fail(QNF4_ERR_UNSUPPORTED, "K must be a multiple of 8 and r <= 1024");
+  if (N * K > (1ll << 35)) return fail(QNF4_ERR_UNSUPPORTED, "N * K above 2^35");
+  if (!aligned(workspace, 256) || (merged_out && !aligned(merged_out, 16)) ||
+      (double_quant && !aligned(scale_codes_out, 8)))
+    return fail(QNF4_ERR_UNSUPPORTED, "alignment: workspace 256 B, merged_out and codes 16 B, scale codes 8 B");
+  const size_t need = qlora_merge_workspace_bytes(N, K, double_quant, merged_out ? 1 : 0);
+  if (workspace_bytes < need) return fail(QNF4_ERR_WORKSPACE, "workspace needs %zu bytes", need);
+  qnf4::Codebook cb;
+  if (int rc = get_codebook(codebook, &cb)) return rc;
+  if (int rc = check_arch()) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  uint16_t* merged = merged_out;
+  if (!merged) {
+    merged = reinterpret_cast<uint16_t*>(ws);
+    ws += align_up((size_t)N * (size_t)K * 2, 256);
+  }
+  qnf4::MergeParams mp;
+  memset(&mp, 0, sizeof(mp));
+  mp.cb = cb;
+  mp.codes = codes;
+  mp.scale_codes = scale_codes;
+  mp.scales = scales;
+  mp.mean = mean;
+  mp.scale_fp32 = double_quant ? 0 : 1;
+  mp.N = N;
+  mp.K = K;
+  mp.A = A;
+  mp.B = B;
+  mp.r = r;
+  mp.s = (double)s;
+  mp.out = merged;
+  cudaError_t e = qnf4::launch_merge_dense(mp, st);
+  if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+  const int64_t numel = N * K, nb = (numel + 63) / 64;
+  float* absmax = double_quant ? reinterpret_cast<float*>(ws) : nullptr;
+  double* gsum = double_quant ? reinterpret_cast<double*>(ws + align_up((size_t)nb * 4, 256)) : nullptr;
+  return quantize_impl(merged, numel, codebook, double_quant, codes_out, scale_codes_out, scales_out, mean_out, absmax,
+                       gsum, st);
 }
 
 size_t qlora_linear_fwd_workspace_bytes(int64_t M, int64_t K, int64_t N, int r) {
@@ -475,9 +633,19 @@ int qlora_linear_fwd(const uint16_t* x, int64_t M, int64_t K, int64_t N, const u
                      const uint8_t* scale_codes, const float* c2, const float* mean, const uint16_t* A,
                      const uint16_t* B, int r, float s, uint16_t* y, float* t_saved, void* workspace,
                      size_t workspace_bytes, void* stream) {
+  return qlora_linear_fwd_ex(x, M, K, N, QNF4_CODEBOOK_NF4, 1, codes, scale_codes, c2, mean, A, B, r, s, y, t_saved,
+                             workspace, workspace_bytes, stream);
+}
+
+int qlora_linear_fwd_ex(const uint16_t* x, int64_t M, int64_t K, int64_t N, int codebook, int double_quant,
+                        const uint8_t* codes, const uint8_t* scale_codes, const float* c2, const float* mean,
+                        const uint16_t* A, const uint16_t* B, int r, float s, uint16_t* y, float* t_saved,
+                        void* workspace, size_t workspace_bytes, void* stream) {
   g_last_error.clear();
-  if (!x || !codes || !scale_codes || !c2 || !mean || !A || !B || !y || !t_saved || !workspace)
-    return fail(QNF4_ERR_INVALID, "NULL pointer");
+  if (!x || !A || !B || !y || !t_saved || !workspace) return fail(QNF4_ERR_INVALID, "NULL pointer");
+  if (int rc = check_format(double_quant, codes, scale_codes, c2, mean)) return rc;
+  qnf4::Codebook cb;
+  if (int rc = get_codebook(codebook, &cb)) return rc;
   LinearShape sh{M, K, N, r};
   if (int rc = check_linear_shape(sh)) return rc;
   if (!aligned(x, 16) || !aligned(A, 16) || !aligned(B, 16) || !aligned(y, 16) || !aligned(codes, 16) ||
@@ -515,7 +683,7 @@ int qlora_linear_fwd(const uint16_t* x, int64_t M, int64_t K, int64_t N, const u
     if (int rc = make_map(&gp.maps[3], w.thi, true, r, M, (uint64_t)r * 2, 64, bbox)) return rc;
     if (int rc = make_map(&gp.maps[4], w.tlo, true, r, M, (uint64_t)r * 2, 64, bbox)) return rc;
     gp.b_box_rows = bbox;
-    nf4_operand(gp, codes, scale_codes, c2, mean, N, K);
+    nf4_operand(gp, cb, double_quant, codes, scale_codes, c2, mean, N, K);
     gp.nseg = 3;
     gp.seg[0] = qnf4::GemmSeg{kblocks(K), k16_last(K), qnf4::kANf4K, 0, 1, 0, 0, 0};
     gp.seg[1] = qnf4::GemmSeg{kblocks(r), k16_last(r), qnf4::kATmaK, 2, 3, 0, 0, 0};
@@ -582,9 +750,20 @@ int qlora_linear_bwd(const uint16_t* dY, const uint16_t* x, const float* t_saved
                      const uint8_t* codes, const uint8_t* scale_codes, const float* c2, const float* mean,
                      const uint16_t* A, const uint16_t* B, int r, float s, uint16_t* dX, uint16_t* dA,
                      uint16_t* dB, void* workspace, size_t workspace_bytes, void* stream) {
+  return qlora_linear_bwd_ex(dY, x, t_saved, M, K, N, QNF4_CODEBOOK_NF4, 1, codes, scale_codes, c2, mean, A, B, r, s,
+                             dX, dA, dB, workspace, workspace_bytes, stream);
+}
+
+int qlora_linear_bwd_ex(const uint16_t* dY, const uint16_t* x, const float* t_saved, int64_t M, int64_t K, int64_t N,
+                        int codebook, int double_quant, const uint8_t* codes, const uint8_t* scale_codes,
+                        const float* c2, const float* mean, const uint16_t* A, const uint16_t* B, int r, float s,
+                        uint16_t* dX, uint16_t* dA, uint16_t* dB, void* workspace, size_t workspace_bytes,
+                        void* stream) {
   g_last_error.clear();
-  if (!dY || !x || !t_saved || !codes || !scale_codes || !c2 || !mean || !A || !B || !dA || !dB || !workspace)
-    return fail(QNF4_ERR_INVALID, "NULL pointer");
+  if (!dY || !x || !t_saved || !A || !B || !dA || !dB || !workspace) return fail(QNF4_ERR_INVALID, "NULL pointer");
+  if (int rc = check_format(double_quant, codes, scale_codes, c2, mean)) return rc;
+  qnf4::Codebook cb;
+  if (int rc = get_codebook(codebook, &cb)) return rc;
   LinearShape sh{M, K, N, r};
   if (int rc = check_linear_shape(sh)) return rc;
   if (!aligned(dY, 16) || !aligned(x, 16) || !aligned(A, 16) || !aligned(B, 16) || !aligned(codes, 16) ||
@@ -632,7 +811,7 @@ int qlora_linear_bwd(const uint16_t* dY, const uint16_t* x, const float* t_saved
     if (int rc = make_map(&gp.maps[3], w.uhi, true, r, M, (uint64_t)r * 2, 64, bbox)) return rc;
     if (int rc = make_map(&gp.maps[4], w.ulo, true, r, M, (uint64_t)r * 2, 64, bbox)) return rc;
     gp.b_box_rows = bbox;
-    nf4_operand(gp, codes, scale_codes, c2, mean, N, K);
+    nf4_operand(gp, cb, double_quant, codes, scale_codes, c2, mean, N, K);
     gp.nseg = 3;
     gp.seg[0] = qnf4::GemmSeg{kblocks(N), k16_last(N), qnf4::kANf4MN, 0, 1, 0, 0, 0};
     gp.seg[1] = qnf4::GemmSeg{kblocks(r), k16_last(r), qnf4::kATmaMN, 2, 3, 0, 0, 0};

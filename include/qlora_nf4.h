@@ -173,6 +173,81 @@ int qlora_linear_bwd(const uint16_t* dY, const uint16_t* x, const float* t_saved
                      uint16_t* dB, void* workspace, size_t workspace_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------------------
+ * Other 16-level code books and single-level (no double quantization) scales.
+ * [T] section 1 (standard INT4: 16 equally spaced levels over [-c, +c]) and section 3
+ * (single blockwise quantization: an fp32 absmax per block of 64, 4 + 32/64 = 4.5 bits per
+ * weight); dmarx anthology sota-230 (the data types compared: Int4, Float4 (E2M1), NF4 + DQ).
+ *
+ * codebook:
+ *   QNF4_CODEBOOK_NF4       the NF4 levels (the default of every other call);
+ *   QNF4_CODEBOOK_FP4_E2M1  the 16 values of the 4-bit float E2M1 (0, 0.5, 1, 1.5, 2, 3, 4, 6,
+ *                           both signs, both zeros) divided by 6, sorted; code j is the j-th
+ *                           value in increasing order (-0 is code 7, +0 code 8), not the E2M1
+ *                           bit pattern;
+ *   QNF4_CODEBOOK_INT4      -1 + 2 j / 15 for j = 0 .. 15.
+ * Each level is the nearest fp32 to its exact value.  A weight takes the code of the nearest
+ * level (an exact tie goes to the lower code; for E2M1 a normalised value of exactly 0 codes
+ * to -0 and any positive one below 1/24 to +0).
+ *
+ * double_quant = 1: the stored format of nf4_quantize_dq (scale_codes[nb] E4M3, scales =
+ *   c2[ceil(nb/256)], mean[1]).
+ * double_quant = 0: scales = one fp32 absmax per block, float[nb]; scale_codes and mean are
+ *   unused (may be NULL); no workspace is needed (qnf4_quantize_workspace_bytes_ex returns a
+ *   token size and the workspace pointer may be NULL).
+ * Everything else (layouts, alignment, errors, bit-exactness) is as for the NF4 calls above;
+ * the dequantized weight is bf16(fp32(level[code] * s_b)) with s_b the block's scale.  The
+ * linear layer calls take the same workspace sizes as qlora_linear_fwd / _bwd.
+ * ------------------------------------------------------------------------------------- */
+#define QNF4_CODEBOOK_NF4 0
+#define QNF4_CODEBOOK_FP4_E2M1 1
+#define QNF4_CODEBOOK_INT4 2
+size_t qnf4_quantize_workspace_bytes_ex(int64_t numel, int double_quant);
+int qnf4_quantize_ex(const uint16_t* W, int64_t numel, int codebook, int double_quant, uint8_t* codes,
+                     uint8_t* scale_codes, float* scales, float* mean, void* workspace, size_t workspace_bytes,
+                     void* stream);
+int qnf4_dequant_ex(const uint8_t* codes, int codebook, int double_quant, const uint8_t* scale_codes,
+                    const float* scales, const float* mean, int64_t numel, uint16_t* W_out, void* stream);
+int qlora_linear_fwd_ex(const uint16_t* x, int64_t M, int64_t K, int64_t N, int codebook, int double_quant,
+                        const uint8_t* codes, const uint8_t* scale_codes, const float* scales, const float* mean,
+                        const uint16_t* A, const uint16_t* B, int r, float s, uint16_t* y, float* t_saved,
+                        void* workspace, size_t workspace_bytes, void* stream);
+int qlora_linear_bwd_ex(const uint16_t* dY, const uint16_t* x, const float* t_saved, int64_t M, int64_t K, int64_t N,
+                        int codebook, int double_quant, const uint8_t* codes, const uint8_t* scale_codes,
+                        const float* scales, const float* mean, const uint16_t* A, const uint16_t* B, int r, float s,
+                        uint16_t* dX, uint16_t* dA, uint16_t* dB, void* workspace, size_t workspace_bytes,
+                        void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * Adapter merge and re-quantization.  [T] "Engineering Limitations" (full-rank updates need
+ * the adapters dequantized and merged into 16-bit precision); [V] (merging / re-quantizing
+ * adapters is a deployment step).
+ *
+ *   W''[n][k] = bf16( W'[n][k] + s * sum_j B[n][j] A[j][k] ),   then W'' is quantized again.
+ *
+ * The rank-r sum is formed in float64, term by term in index order j = 0 .. r-1; then
+ * t = float64(s * sum), v = float64(W' + t), and W'' is v rounded once to the nearest bf16
+ * (ties to even).  W' is the dequantized base (as nf4_dequant / qnf4_dequant_ex produce it).
+ * The result is then coded exactly as qnf4_quantize_ex codes a bf16 weight, with the same
+ * code book and format as the input (codebook, double_quant as in qnf4_quantize_ex).
+ *
+ *   codes, scale_codes, scales, mean          : the stored base W' [N][K], read only
+ *   A : bf16[r][K]    B : bf16[N][r]    s : the LoRA scale alpha / r
+ *   codes_out, scale_codes_out, scales_out, mean_out : the re-quantized W'' (may not alias the
+ *                                               inputs), written
+ *   merged_out : bf16[N][K] receiving W'' itself (16-byte aligned), or NULL to keep it in the
+ *                workspace
+ *   workspace  : qlora_merge_workspace_bytes(N, K, double_quant, merged_out != NULL) bytes,
+ *                256-byte aligned
+ * Requirements: K % 8 == 0, r <= 1024, N * K <= 2^35.
+ * ------------------------------------------------------------------------------------- */
+size_t qlora_merge_workspace_bytes(int64_t N, int64_t K, int double_quant, int merged_out_given);
+int qlora_merge_requantize(const uint8_t* codes, const uint8_t* scale_codes, const float* scales, const float* mean,
+                           int64_t N, int64_t K, int codebook, int double_quant, const uint16_t* A, const uint16_t* B,
+                           int r, float s, uint8_t* codes_out, uint8_t* scale_codes_out, float* scales_out,
+                           float* mean_out, uint16_t* merged_out, void* workspace, size_t workspace_bytes,
+                           void* stream);
+
+/* ---------------------------------------------------------------------------------------
  * Launch plan of one forward / backward call of this shape (host-only, no device work):
  * the number of kernels each call enqueues, and the split factor of the K loop of the
  * fused dequant GEMMs (1 = no split).  Output pointers are HOST pointers and may be NULL.
