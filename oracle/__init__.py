@@ -21,9 +21,10 @@ Sources, cited by page title and section:
   description) -- the Appendix-E lookup example and the storage arithmetic.
 
 Pin status of every function is listed in the module docstrings of
-``oracle.nf4``, ``oracle.linear`` and ``oracle.variants`` (the FP4-E2M1 and INT4 code books,
-single-level quantization without double quantization, adapter merge + re-quantization).  No function is "parity unpinned": each has
+``oracle.nf4``, ``oracle.linear``, ``oracle.variants`` (the FP4-E2M1 and INT4 code books,
+single-level quantization without double quantization, adapter merge + re-quantization) and
+``oracle.adamw`` (the AdamW step of the paged optimizer).  No function is "parity unpinned": each has
 at least one check against the pages or the mathematics in ``tests/``.
 """
 
-from . import nf4, linear, variants  # noqa: F401
+from . import nf4, linear, variants, adamw  # noqa: F401
