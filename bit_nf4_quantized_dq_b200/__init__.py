@@ -21,8 +21,9 @@ from .binding import (  # noqa: F401
     quantize,
     set_timing_events,
 )
+from .paged import PagedAdamW  # noqa: F401
 
 __all__ = [
-    "NF4Tensor", "QNF4Error", "check_device_error", "e4m3_encode", "lib", "library_path", "linear_plan", "merge_requantize", "set_timing_events",
+    "NF4Tensor", "PagedAdamW", "QNF4Error", "check_device_error", "e4m3_encode", "lib", "library_path", "linear_plan", "merge_requantize", "set_timing_events",
     "nf4_dequant", "nf4_quantize_dq", "qlora_linear_bwd", "qlora_linear_fwd", "quantize",
 ]

@@ -49,6 +49,11 @@ SIGNATURES = {
     "qlora_linear_fwd_ex": (c_int, [c_void_p, c_int64, c_int64, c_int64, c_int, c_int, c_void_p, c_void_p,
                                     c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_float, c_void_p, c_void_p,
                                     c_void_p, c_size_t, c_void_p]),
+    "qnf4_paged_alloc": (c_int, [c_size_t, ctypes.POINTER(c_void_p)]),
+    "qnf4_paged_free": (c_int, [c_void_p]),
+    "qnf4_paged_prefetch": (c_int, [c_void_p, c_size_t, c_int, c_void_p]),
+    "qlora_adamw_step": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_float, c_float,
+                                 c_float, c_float, c_float, c_int, c_void_p]),
     "qlora_merge_workspace_bytes": (c_size_t, [c_int64, c_int64, c_int, c_int]),
     "qlora_merge_requantize": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_int, c_int,
                                        c_void_p, c_void_p, c_int, c_float, c_void_p, c_void_p, c_void_p, c_void_p,

@@ -13,6 +13,7 @@
 #include "gemm.cuh"
 #include "lowrank.cuh"
 #include "merge.cuh"
+#include "adamw.cuh"
 
 namespace {
 
@@ -561,6 +562,59 @@ int nf4_e4m3_encode(const float* v, int64_t n, uint8_t* out, int mode, void* str
   if (int rc = check_arch()) return rc;
   cudaError_t e = qnf4::launch_e4m3_encode(v, n, out, mode, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "e4m3 launch");
+  return QNF4_OK;
+}
+
+int qnf4_paged_alloc(size_t bytes, void** ptr) {
+  g_last_error.clear();
+  if (!ptr) return fail(QNF4_ERR_INVALID, "NULL pointer");
+  if (bytes == 0) return fail(QNF4_ERR_INVALID, "bytes must be positive");
+  *ptr = nullptr;
+  cudaError_t e = cudaMallocManaged(ptr, bytes, cudaMemAttachGlobal);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMallocManaged");
+  return QNF4_OK;
+}
+
+int qnf4_paged_free(void* ptr) {
+  g_last_error.clear();
+  if (!ptr) return QNF4_OK;
+  cudaError_t e = cudaFree(ptr);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFree of managed memory");
+  return QNF4_OK;
+}
+
+int qnf4_paged_prefetch(const void* ptr, size_t bytes, int to_device, void* stream) {
+  g_last_error.clear();
+  if (!ptr || bytes == 0) return fail(QNF4_ERR_INVALID, "NULL pointer or zero size");
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  e = cudaMemPrefetchAsync(ptr, bytes, to_device ? dev : cudaCpuDeviceId, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemPrefetchAsync");
+  return QNF4_OK;
+}
+
+int qlora_adamw_step(float* param, const uint16_t* grad, float* m, float* v, uint16_t* param_bf16, int64_t n,
+                     float lr, float beta1, float beta2, float eps, float weight_decay, int step, void* stream) {
+  g_last_error.clear();
+  if (!param || !grad || !m || !v) return fail(QNF4_ERR_INVALID, "NULL pointer");
+  if (n <= 0 || step <= 0) return fail(QNF4_ERR_INVALID, "n and step must be positive");
+  if (!(beta1 >= 0.0f && beta1 < 1.0f && beta2 >= 0.0f && beta2 < 1.0f))
+    return fail(QNF4_ERR_INVALID, "betas must lie in [0, 1)");
+  if (!aligned(param, 16) || !aligned(m, 16) || !aligned(v, 16) || !aligned(grad, 8) ||
+      (param_bf16 && !aligned(param_bf16, 8)))
+    return fail(QNF4_ERR_UNSUPPORTED, "alignment: param, m, v 16 B; grad and param_bf16 8 B");
+  if (int rc = check_arch()) return rc;
+  qnf4::AdamWArgs a;
+  a.lr = lr;
+  a.b1 = beta1;
+  a.b2 = beta2;
+  a.eps = eps;
+  a.wd = weight_decay;
+  a.bc1 = (float)(1.0 - std::pow((double)beta1, (double)step));
+  a.bc2 = (float)(1.0 - std::pow((double)beta2, (double)step));
+  cudaError_t e = qnf4::launch_adamw(param, grad, m, v, param_bf16, n, a, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "adamw launch");
   return QNF4_OK;
 }
 

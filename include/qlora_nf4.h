@@ -11,9 +11,9 @@
  *
  * Conventions for every entry point:
  *  - Every pointer is a DEVICE pointer owned by the caller, except where stated.  The library
- *    never allocates device memory and keeps no state between calls other than the device
- *    error word (see qnf4_device_error) and the static scratch array of
- *    nf4_quantize_dq_noalloc.
+ *    allocates no device memory (except qnf4_paged_alloc, on request, for optimizer states) and
+ *    keeps no state between calls other than the device error word (see qnf4_device_error) and
+ *    the static scratch array of nf4_quantize_dq_noalloc.
  *  - bf16 tensors are passed as uint16_t bit patterns, row-major, densely packed.
  *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every call is
  *    stream-ordered and asynchronous: it returns after enqueueing its kernels.  Device-side
@@ -246,6 +246,31 @@ int qlora_merge_requantize(const uint8_t* codes, const uint8_t* scale_codes, con
                            int r, float s, uint8_t* codes_out, uint8_t* scale_codes_out, float* scales_out,
                            float* mean_out, uint16_t* merged_out, void* workspace, size_t workspace_bytes,
                            void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * Paged AdamW on the LoRA parameters.  [T] section 5 (the AdamW states of the adapters live in
+ * CUDA unified memory, which the driver evicts to host RAM under memory pressure and pages back
+ * for the optimizer step); [E] step 6.
+ *
+ * qlora_adamw_step: one AdamW step with decoupled weight decay on n parameters:
+ *   m = b1 m + (1 - b1) g,  v = b2 v + (1 - b2) g^2,
+ *   p = p - lr ( (m / (1 - b1^step)) / (sqrt(v / (1 - b2^step)) + eps) + weight_decay p ).
+ *   param, m, v : float[n], updated in place (16-byte aligned);  grad : bf16[n] (8-byte aligned);
+ *   param_bf16  : bf16[n] receiving the updated parameters rounded to bf16, or NULL.
+ *   step is 1-based.  fp32 arithmetic with IEEE division and square root.  Any of the pointers
+ *   may be managed memory (qnf4_paged_alloc); such memory should be on the device
+ *   (qnf4_paged_prefetch) when the step runs, or the driver migrates it page by page.
+ *
+ * qnf4_paged_alloc / qnf4_paged_free: CUDA managed memory for optimizer states (these two are
+ *   the library's only allocating calls).  `ptr` is a HOST pointer receiving the address.
+ * qnf4_paged_prefetch: stream-ordered migration of a managed range to the current device
+ *   (to_device = 1) or to host memory (to_device = 0: eviction).
+ * ------------------------------------------------------------------------------------- */
+int qnf4_paged_alloc(size_t bytes, void** ptr);
+int qnf4_paged_free(void* ptr);
+int qnf4_paged_prefetch(const void* ptr, size_t bytes, int to_device, void* stream);
+int qlora_adamw_step(float* param, const uint16_t* grad, float* m, float* v, uint16_t* param_bf16, int64_t n,
+                     float lr, float beta1, float beta2, float eps, float weight_decay, int step, void* stream);
 
 /* ---------------------------------------------------------------------------------------
  * Launch plan of one forward / backward call of this shape (host-only, no device work):
