@@ -688,12 +688,72 @@ def rows_robust(L, dev, peaks, peak):
             "note": "fwd + bwd through the Python binding (allocating outputs); M <= 16 is HBM-bound"}
 
 
+def rows_variants(dev, peaks, peak):
+    """Code books and scale formats on the 13B q linear (5120 x 5120, 8192 tokens, r = 64):
+    stored bits per weight, quantize / dequant GB/s (algorithmic bytes: bf16 in, codes and
+    scales out, or the reverse) and the fused forward + backward TFLOP/s; then the adapter
+    merge + re-quantization and one paged AdamW step over the block's adapters."""
+    import torch
+    import synth
+    import bit_nf4_quantized_dq_b200 as q
+    N = K = 5120
+    M = M_TOKENS
+    W = synth.normal_bf16((N, K), 0.02, 3000, device=str(dev))
+    inp = synth.linear_inputs(M, N, K, R, 3000, device=str(dev))
+    x, A, B, dY = inp["x"], inp["A"], inp["B"], inp["dY"]
+    s = ALPHA / R
+    L = q.lib()
+    wsf = torch.empty(max(256, L.qlora_linear_fwd_workspace_bytes(M, K, N, R)), dtype=torch.uint8, device=dev)
+    wsb = torch.empty(max(256, L.qlora_linear_bwd_workspace_bytes(M, K, N, R)), dtype=torch.uint8, device=dev)
+    out = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+    numel = N * K
+    points = []
+    for cb in ("nf4", "fp4_e2m1", "int4"):
+        for dq in (True, False):
+            Q = q.quantize(W, codebook=cb, double_quant=dq)
+            bits = Q.nbytes() * 8 / numel
+            codec_bytes = numel * (2 + bits / 8)
+            tq = _time_calls(lambda: q.quantize(W, codebook=cb, double_quant=dq), 10)
+            td = _time_calls(lambda: q.nf4_dequant(Q, out=out), 20)
+
+            def fb():
+                y, t = q.qlora_linear_fwd(x, Q, A, B, s, workspace=wsf)
+                q.qlora_linear_bwd(dY, x, t, Q, A, B, s, workspace=wsb)
+
+            tl = _time_calls(fb, 5)
+            fl = linear_flops(M, N, K, R)
+            points.append({"codebook": cb, "double_quant": dq, "bits_per_weight": bits,
+                           "quantize_gbs": codec_bytes / (tq * 1e6), "dequant_gbs": codec_bytes / (td * 1e6),
+                           "dequant_frac_hbm": codec_bytes / (td * 1e6) / peaks["hbm_gbs"],
+                           "linear_fwd_bwd_tflops": fl / (tl * 1e9), "linear_frac": fl / (tl * 1e9) / peak})
+    Q = q.nf4_quantize_dq(W)
+    Ab, Bb = A, B * 20
+    tm = _time_calls(lambda: q.merge_requantize(Q, Ab, Bb, s), 5)
+    merge = {"shape": "5120x5120 r=64 NF4+DQ", "ms": tm, "gweights_per_s": numel / (tm * 1e6),
+             "note": "W'' = bf16(W' + s B A), float64 rank-r sum, then re-quantized; float64-bound"}
+    lins = linears()
+    sizes = [R * l.K + l.N * R for l in lins]
+    params = [torch.zeros(n, dtype=torch.float32, device=dev) for n in sizes]
+    grads = [torch.zeros(n, dtype=torch.bfloat16, device=dev) for n in sizes]
+    opt = q.PagedAdamW(params, None, lr=1e-4, paged=True)
+    ta = _time_calls(lambda: opt.step(grads), 10)
+    nparam = sum(sizes)
+    opt.close()
+    adam = {"params": nparam, "ms": ta, "gbs": nparam * 22 / (ta * 1e6),
+            "note": "paged AdamW step over the 13B block's adapters (states in managed memory, paged in each step);"
+                    " 22 B per parameter (fp32 p, m, v read and written, bf16 g read)"}
+    return {"variants_13b_q": points, "merge_13b_q": merge, "adamw_13b_block": adam}
+
+
 def extra_rows(args, L, dev, peaks, peak):
     import torch
     torch.cuda.empty_cache()
-    return {"llama7b_512": rows_llama7b_512(L, dev, peak),
+    rows = {"llama7b_512": rows_llama7b_512(L, dev, peak),
             "stack65b": rows_stack65b(L, dev, peaks["hbm_gbs"], args.stack_layers),
             "robust": rows_robust(L, dev, peaks, peak)}
+    torch.cuda.empty_cache()
+    rows.update(rows_variants(dev, peaks, peak))
+    return rows
 
 
 # ------------------------------------------------------------------------------------------
