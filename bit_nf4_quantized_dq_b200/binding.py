@@ -22,6 +22,7 @@ c_int64 = ctypes.c_int64
 c_int = ctypes.c_int
 c_size_t = ctypes.c_size_t
 c_float = ctypes.c_float
+c_double = ctypes.c_double
 
 # name -> (restype, argtypes); mirrors include/qlora_nf4.h
 SIGNATURES = {
@@ -52,8 +53,8 @@ SIGNATURES = {
     "qnf4_paged_alloc": (c_int, [c_size_t, ctypes.POINTER(c_void_p)]),
     "qnf4_paged_free": (c_int, [c_void_p]),
     "qnf4_paged_prefetch": (c_int, [c_void_p, c_size_t, c_int, c_void_p]),
-    "qlora_adamw_step": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_float, c_float,
-                                 c_float, c_float, c_float, c_int, c_void_p]),
+    "qlora_adamw_step": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_double, c_double,
+                                 c_double, c_double, c_double, c_int, c_void_p]),
     "qlora_merge_workspace_bytes": (c_size_t, [c_int64, c_int64, c_int, c_int]),
     "qlora_merge_requantize": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_int, c_int,
                                        c_void_p, c_void_p, c_int, c_float, c_void_p, c_void_p, c_void_p, c_void_p,

@@ -13,13 +13,16 @@
 
 namespace qnf4 {
 
+// Every constant is the fp32 rounding of a value the host formed in double: in particular
+// omb1 = 1 - b1 and omb2 = 1 - b2 (forming 1 - b2 in fp32 from an fp32 b2 = 0.999 would miss
+// the true 0.001 by about 1.3e-5 relative).
 struct AdamWArgs {
-  float lr, b1, b2, eps, wd, bc1, bc2;
+  float lr, b1, omb1, b2, omb2, eps, wd, bc1, bc2;
 };
 
 __device__ __forceinline__ void adamw_one(float& p, float g, float& m, float& v, const AdamWArgs& a) {
-  m = __fmaf_rn(a.b1, m, __fmul_rn(1.0f - a.b1, g));
-  v = __fmaf_rn(a.b2, v, __fmul_rn(1.0f - a.b2, __fmul_rn(g, g)));
+  m = __fmaf_rn(a.b1, m, __fmul_rn(a.omb1, g));
+  v = __fmaf_rn(a.b2, v, __fmul_rn(a.omb2, __fmul_rn(g, g)));
   const float mhat = __fdiv_rn(m, a.bc1);
   const float vhat = __fdiv_rn(v, a.bc2);
   const float upd = __fadd_rn(__fdiv_rn(mhat, __fadd_rn(__fsqrt_rn(vhat), a.eps)), __fmul_rn(a.wd, p));

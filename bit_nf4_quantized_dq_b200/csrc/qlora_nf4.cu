@@ -595,24 +595,27 @@ int qnf4_paged_prefetch(const void* ptr, size_t bytes, int to_device, void* stre
 }
 
 int qlora_adamw_step(float* param, const uint16_t* grad, float* m, float* v, uint16_t* param_bf16, int64_t n,
-                     float lr, float beta1, float beta2, float eps, float weight_decay, int step, void* stream) {
+                     double lr, double beta1, double beta2, double eps, double weight_decay, int step,
+                     void* stream) {
   g_last_error.clear();
   if (!param || !grad || !m || !v) return fail(QNF4_ERR_INVALID, "NULL pointer");
   if (n <= 0 || step <= 0) return fail(QNF4_ERR_INVALID, "n and step must be positive");
-  if (!(beta1 >= 0.0f && beta1 < 1.0f && beta2 >= 0.0f && beta2 < 1.0f))
+  if (!(beta1 >= 0.0 && beta1 < 1.0 && beta2 >= 0.0 && beta2 < 1.0))
     return fail(QNF4_ERR_INVALID, "betas must lie in [0, 1)");
   if (!aligned(param, 16) || !aligned(m, 16) || !aligned(v, 16) || !aligned(grad, 8) ||
       (param_bf16 && !aligned(param_bf16, 8)))
     return fail(QNF4_ERR_UNSUPPORTED, "alignment: param, m, v 16 B; grad and param_bf16 8 B");
   if (int rc = check_arch()) return rc;
   qnf4::AdamWArgs a;
-  a.lr = lr;
-  a.b1 = beta1;
-  a.b2 = beta2;
-  a.eps = eps;
-  a.wd = weight_decay;
-  a.bc1 = (float)(1.0 - std::pow((double)beta1, (double)step));
-  a.bc2 = (float)(1.0 - std::pow((double)beta2, (double)step));
+  a.lr = (float)lr;
+  a.b1 = (float)beta1;
+  a.omb1 = (float)(1.0 - beta1);
+  a.b2 = (float)beta2;
+  a.omb2 = (float)(1.0 - beta2);
+  a.eps = (float)eps;
+  a.wd = (float)weight_decay;
+  a.bc1 = (float)(1.0 - std::pow(beta1, (double)step));
+  a.bc2 = (float)(1.0 - std::pow(beta2, (double)step));
   cudaError_t e = qnf4::launch_adamw(param, grad, m, v, param_bf16, n, a, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "adamw launch");
   return QNF4_OK;

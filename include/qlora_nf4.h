@@ -257,7 +257,10 @@ int qlora_merge_requantize(const uint8_t* codes, const uint8_t* scale_codes, con
  *   p = p - lr ( (m / (1 - b1^step)) / (sqrt(v / (1 - b2^step)) + eps) + weight_decay p ).
  *   param, m, v : float[n], updated in place (16-byte aligned);  grad : bf16[n] (8-byte aligned);
  *   param_bf16  : bf16[n] receiving the updated parameters rounded to bf16, or NULL.
- *   step is 1-based.  fp32 arithmetic with IEEE division and square root.  Any of the pointers
+ *   step is 1-based.  The hyper-parameters are doubles: the kernel uses lr, b1, 1 - b1, b2,
+ *   1 - b2, eps, weight_decay and the two bias corrections each rounded once to fp32 from the
+ *   value formed in double (so 1 - b2 = 0.001 is not lost to an fp32 b2).  fp32 arithmetic
+ *   with IEEE division and square root.  Any of the pointers
  *   may be managed memory (qnf4_paged_alloc); such memory should be on the device
  *   (qnf4_paged_prefetch) when the step runs, or the driver migrates it page by page.
  *
@@ -270,7 +273,8 @@ int qnf4_paged_alloc(size_t bytes, void** ptr);
 int qnf4_paged_free(void* ptr);
 int qnf4_paged_prefetch(const void* ptr, size_t bytes, int to_device, void* stream);
 int qlora_adamw_step(float* param, const uint16_t* grad, float* m, float* v, uint16_t* param_bf16, int64_t n,
-                     float lr, float beta1, float beta2, float eps, float weight_decay, int step, void* stream);
+                     double lr, double beta1, double beta2, double eps, double weight_decay, int step,
+                     void* stream);
 
 /* ---------------------------------------------------------------------------------------
  * Launch plan of one forward / backward call of this shape (host-only, no device work):
