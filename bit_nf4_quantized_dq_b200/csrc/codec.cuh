@@ -82,6 +82,66 @@ __device__ __forceinline__ bool recip_path_ok(float c) {
   return c >= 7.888609052210118e-31f && c <= 1.2676506002282294e+30f;   // 2^-100 .. 2^100
 }
 
+// Two fp32 lanes in one 64-bit register pair, for the sm_100 paired fp32 instructions (each
+// lane is rounded exactly as the scalar instruction would round it).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float f2_lo(uint64_t v) { return __uint_as_float((uint32_t)v); }
+__device__ __forceinline__ float f2_hi(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+
+// Packed bf16 pair -> its two fp32 values (exact), as one register pair.
+__device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t u) {
+  return f2_pack(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
+}
+
+// max(|a|, |b|) of each bf16 lane (the sign of the result, the xor of the inputs', is
+// discarded by the caller).  A NaN input gives NaN, so that a block holding one never takes
+// the table path below (whose bucket address is only in range for |n| <= 1).
+__device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ float fmax_nan(float a, float b) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+
+// One bucket-table entry by its 32-bit shared-memory address.
+__device__ __forceinline__ uint2 lds_entry(uint32_t addr) {
+  uint2 v;
+  asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
+}
+
+// Codes of one packed word (two weights) given n for both: bucket index from one fused
+// multiply-add each (1.5 * 2^23 + 16 + 16 n rounds to the integer 16 + round(16 n) in the low
+// mantissa bits, so (bits << 8) is 256 * bucket plus a constant that lane_bias cancels: one
+// shift-add forms the entry's address), then code = base + (n > threshold), the comparison
+// taken from the sign of the correctly rounded threshold - n (zero only when they are equal).
+__device__ __forceinline__ uint32_t codes_of_pair(uint64_t n2, uint32_t lane_bias) {
+  const uint64_t t2 = f2_fma(n2, f2_pack(16.0f, 16.0f), f2_pack(12582928.0f, 12582928.0f));
+  const uint2 e0 = lds_entry(((uint32_t)t2 << 8) + lane_bias);
+  const uint2 e1 = lds_entry(((uint32_t)(t2 >> 32) << 8) + lane_bias);
+  const uint32_t c0 = e0.x + (__float_as_uint(__fsub_rn(__uint_as_float(e0.y), f2_lo(n2))) >> 31);
+  const uint32_t c1 = e1.x + (__float_as_uint(__fsub_rn(__uint_as_float(e1.y), f2_hi(n2))) >> 31);
+  return c0 + (c1 << 4);
+}
+
 // Q-A: one group of 256 blocks (16384 weights, 32 KB of bf16) per CTA iteration; thread t
 // takes block t of the group: eight 16-byte loads (128 contiguous bytes, all in flight before
 // any is used), absmax over its 64 weights, the correctly rounded n = w / absmax, the nearest
@@ -138,6 +198,13 @@ constexpr int kQGroupWarps = 16;                      // warps coding one group 
 constexpr int kQConsumerWarps = kQGroupWarps;
 constexpr int kQThreads = 32 * (kQConsumerWarps + 1);
 constexpr int kQSmemBytes = kQStages * kQStageBytes + 1024;
+// Warp sums of a group are handed to thread 0 through a ring of kQSumSlots slots, each with an
+// mbarrier that the group's warps arrive on; thread 0 forms a group's float64 sum one group
+// later, so no warp waits for the others.  A warp can run at most kQStages groups ahead of the
+// slowest one (a stage is reloaded only after every warp released it), so slot i % kQSumSlots
+// is not rewritten, and its barrier not two phases ahead, while thread 0 still reads group i.
+constexpr int kQSumSlots = 6;
+static_assert(kQSumSlots >= kQStages + 3 && kQSumSlots <= 8, "sum ring too short for the pipeline depth");
 
 struct QuantParams {
   CUtensorMap w_map;          // W as [nb_full][64] bf16, box 64 x 256, 128-byte swizzle
@@ -153,8 +220,8 @@ __global__ void __launch_bounds__(kQThreads, 2) nf4_quant_stream_kernel(const __
   extern __shared__ uint8_t qsmem_dyn[];
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(qsmem_dyn) + 1023) & ~uintptr_t(1023));
   __shared__ BucketEntry tab[33][32];
-  __shared__ uint64_t full[kQStages], empty[kQStages];
-  __shared__ double warp_sum[2][kQGroupWarps];
+  __shared__ uint64_t full[kQStages], empty[kQStages], psum[kQSumSlots];
+  __shared__ double warp_sum[kQSumSlots][kQGroupWarps];
   __shared__ uint32_t abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -162,6 +229,7 @@ __global__ void __launch_bounds__(kQThreads, 2) nf4_quant_stream_kernel(const __
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kQGroupWarps);
     }
+    for (int s = 0; s < kQSumSlots; ++s) mbar_init(&psum[s], kQGroupWarps);
     abort_flag = 0u;
     mbar_fence_init();
   }
@@ -195,14 +263,30 @@ __global__ void __launch_bounds__(kQThreads, 2) nf4_quant_stream_kernel(const __
     // ------------------------------------------------------------------ consumers
     const int t = threadIdx.x;
     const int r = t >> 1, h = t & 1;          // block of the group, and which half of it
-    int parity = 0;
-    for (int64_t i = 0; i < n_local; ++i, parity ^= 1) {
-      const int s = (int)(i % kQStages);
-      const uint32_t ph = (uint32_t)(i / kQStages) & 1u;
+    // tab[v][lane] sits at tab + 256 v + 8 lane; the bucket's float bits shifted left by 8
+    // carry 256 v plus 0x40000000 (mod 2^32), which the bias removes
+    const uint32_t lane_bias = smem_u32(&tab[0][lane]) - 0x40000000u;
+    int s = 0;
+    uint32_t ph = 0;
+    // sum-ring position: slot in bits 0-2, phase parity in bit 3
+    uint32_t sp = 0, prev_sp = 0;
+    // thread 0: the float64 sum of group i from its sixteen warp sums (adjacent-pair tree)
+    auto group_sum = [&](int64_t i, uint32_t at) -> bool {
+      const int sl = (int)(at & 7u);
+      if (!mbar_wait_thread(&psum[sl], at >> 3, abort_word, kErrWaitGroup)) return false;
+      const double* w = warp_sum[sl];
+      const double q0 = ((w[0] + w[1]) + (w[2] + w[3])) + ((w[4] + w[5]) + (w[6] + w[7]));
+      const double q1 = ((w[8] + w[9]) + (w[10] + w[11])) + ((w[12] + w[13]) + (w[14] + w[15]));
+      p.gsum[blockIdx.x + i * gridDim.x] = q0 + q1;
+      return true;
+    };
+    const bool sums = warp == 0 && p.gsum != nullptr;   // no group sums without double quantization
+    int64_t i = 0;
+    for (; i < n_local; ++i) {
       const int64_t g = blockIdx.x + i * gridDim.x;
       const int64_t b = g * kB2 + r;
-      // a warp whose wait gave up still takes part in the group barrier below, so that the
-      // other warps of its group are not left waiting there; all of them leave after it
+      // a warp whose wait gave up still hands in its (zero) warp sum below, so that thread 0
+      // is not left waiting for it; all warps leave at the abort check after that
       bool ok = true;
       uint4 v[4];
       if (p.nb_full > 0) {
@@ -216,34 +300,40 @@ __global__ void __launch_bounds__(kQThreads, 2) nf4_quant_stream_kernel(const __
       const bool whole = ok && b < p.nb_full;
       float m = 0.0f;
       if (ok && p.nb_full > 0) {
-        // every loaded word enters the absmax, so the stage's data are in registers before the
-        // stage is handed back for the next load
+        // every loaded word enters the absmax (bf16 pairs, max of magnitudes, exact), so the
+        // stage's data are in registers before the stage is handed back for the next load
+        uint32_t a2[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint32_t u[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            m = fmaxf(m, fabsf(__uint_as_float(u[k] << 16)));
-            m = fmaxf(m, fabsf(__uint_as_float(u[k] & 0xFFFF0000u)));
-          }
-        }
+        for (int j = 0; j < 4; ++j) a2[j] = bf16x2_absmax(bf16x2_absmax(v[j].x, v[j].y), bf16x2_absmax(v[j].z, v[j].w));
+        const uint32_t am = bf16x2_absmax(bf16x2_absmax(a2[0], a2[1]), bf16x2_absmax(a2[2], a2[3]));
+        m = fmax_nan(__uint_as_float((am << 16) & 0x7FFF0000u), __uint_as_float(am & 0x7FFF0000u));
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
         if (!whole) m = 0.0f;
       }
+      if (++s == kQStages) {
+        s = 0;
+        ph ^= 1u;
+      }
       if (!whole && ok && b < p.nb && h == 0) {
         m = quant_block_global(p.W, b, p.numel, tab, lane, p.codes32, p.absmax);
       }
-      m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));   // join the two halves of each block
+      // join the two halves of each block (a NaN in either half reaches both)
+      m = fmax_nan(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
       double sum = (double)m;
 #pragma unroll
       for (int off = 2; off < 32; off <<= 1) sum = sum + __shfl_xor_sync(0xFFFFFFFFu, sum, off);
-      if (lane == 0) warp_sum[parity][warp] = sum;
+      if (lane == 0) {
+        warp_sum[sp & 7u][warp] = sum;
+        mbar_arrive(&psum[sp & 7u]);   // release: the sum is visible to thread 0 after its wait
+      }
       if (whole) {
         if (h == 0) p.absmax[b] = m;
         uint4* dst = reinterpret_cast<uint4*>(p.codes32 + b * 8) + h;
+        // table path: 2^-100 <= m <= 2^100 and no NaN in the block, so every |n| <= 1
         if (m > 0.0f && recip_path_ok(m)) {
           const Recip2 y = recip2(m);
+          const uint64_t yhi = f2_pack(y.hi, y.hi), ylo = f2_pack(y.lo, y.lo);
           uint32_t packed[4];
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
@@ -251,8 +341,10 @@ __global__ void __launch_bounds__(kQThreads, 2) nf4_quant_stream_kernel(const __
             uint32_t pk = 0u;
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-              pk += nearest_code(div_rn_recip2(__uint_as_float(u[k] << 16), y), tab, lane) << (8 * k);
-              pk += nearest_code(div_rn_recip2(__uint_as_float(u[k] & 0xFFFF0000u), y), tab, lane) << (8 * k + 4);
+              // n = RN(w / m) for both weights of the word (the reciprocal-pair quotient)
+              const uint64_t w2 = bf16x2_to_f2(u[k]);
+              const uint64_t n2 = f2_fma(w2, yhi, f2_mul(w2, ylo));
+              pk += codes_of_pair(n2, lane_bias) << (8 * k);
             }
             packed[j] = pk;
           }
@@ -263,17 +355,17 @@ __global__ void __launch_bounds__(kQThreads, 2) nf4_quant_stream_kernel(const __
           *dst = make_uint4(0x77777777u, 0x77777777u, 0x77777777u, 0x77777777u);   // all-zero block: level 7
         }
       }
-      // one barrier of the group's warps per group: the warp sums alternate between two
-      // buffers, so thread 0 reads this group's while the warps fill the other one
-      asm volatile("bar.sync 1, %0;" ::"r"(32 * kQGroupWarps) : "memory");
-      if (*abort_word) break;
-      if (t == 0 && p.gsum != nullptr) {   // no group sums without double quantization
-        const double* w = warp_sum[parity];
-        const double q0 = ((w[0] + w[1]) + (w[2] + w[3])) + ((w[4] + w[5]) + (w[6] + w[7]));
-        const double q1 = ((w[8] + w[9]) + (w[10] + w[11])) + ((w[12] + w[13]) + (w[14] + w[15]));
-        p.gsum[g] = q0 + q1;
+      if (sums && i > 0) {
+        // lane 0 waits; the whole warp takes the outcome, so it stays converged
+        bool done = true;
+        if (lane == 0) done = group_sum(i - 1, prev_sp);
+        if (!__shfl_sync(0xFFFFFFFFu, (int)done, 0)) break;
       }
+      prev_sp = sp;
+      sp = (sp & 7u) == kQSumSlots - 1 ? (sp & 8u) ^ 8u : sp + 1u;
+      if (__any_sync(0xFFFFFFFFu, *abort_word != 0u)) break;
     }
+    if (sums && lane == 0 && i == n_local && n_local > 0) group_sum(n_local - 1, prev_sp);
   }
   // let the dependent double-quantization kernel start its launch while this grid drains
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -282,26 +374,31 @@ __global__ void __launch_bounds__(kQThreads, 2) nf4_quant_stream_kernel(const __
 // ---------------------------------------------------------------------------------------
 // Q-B: double quantization.  Every CTA first forms the mean itself (so no other launch or
 // grid-wide wait is needed): the float64 group sums, zero-padded, are reduced by the same
-// adjacent-pair tree in aligned chunks of 2048 (eight per thread in registers, then the warp
-// butterfly, then the eight warp sums), then the chunk sums (zero-padded to a power of two)
-// by one warp.  Zero padding leaves every partial sum unchanged, so this equals the tree over
-// the sums padded to the next power of two.  mean = fp32(sum / nb).  Then one warp per group
-// of 256 absmax values: d = fp32(c - mean), c2 = max |d|, code = E4M3(fp32(d / c2)).
+// adjacent-pair tree in aligned chunks of 8192 (eight per thread in registers, then the warp
+// butterfly, then the 32 warp sums by one more butterfly), then the chunk sums (zero-padded to
+// a power of two) by one warp.  Zero padding leaves every partial sum unchanged, so this
+// equals the tree over the sums padded to the next power of two.  mean = fp32(sum / nb).  A
+// group count up to 8192 (numel up to 2^27) takes one pass, so one round trip to memory.
+// Then one warp per group of 256 absmax values: d = fp32(c - mean), c2 = max |d|,
+// code = E4M3(fp32(d / c2)).
 // ---------------------------------------------------------------------------------------
-constexpr int kMaxMeanChunks = 1024;           // 2^21 groups: numel up to 2^35
+constexpr int kDqThreads = 1024;
+constexpr int kDqWarps = kDqThreads / 32;
+constexpr int kDqChunk = 8 * kDqThreads;       // group sums per pass
+constexpr int kMaxMeanChunks = 1024;           // 2^23 groups: numel up to 2^37
 
-__global__ void __launch_bounds__(256) dq_mean_groups_kernel(const float* __restrict__ absmax,
-                                                             const double* __restrict__ gsum, int64_t nb,
-                                                             int64_t ng, float* __restrict__ mean_out,
-                                                             uint8_t* __restrict__ scale_codes,
-                                                             float* __restrict__ c2, int sw_encode) {
-  __shared__ double warp_sum[8];
+__global__ void __launch_bounds__(kDqThreads, 1) dq_mean_groups_kernel(const float* __restrict__ absmax,
+                                                                    const double* __restrict__ gsum, int64_t nb,
+                                                                    int64_t ng, float* __restrict__ mean_out,
+                                                                    uint8_t* __restrict__ scale_codes,
+                                                                    float* __restrict__ c2, int sw_encode) {
+  __shared__ double warp_sum[kDqWarps];
   __shared__ double chunk_sum[kMaxMeanChunks];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   // the quantize kernel's absmax values and group sums are complete and visible after this
   asm volatile("griddepcontrol.wait;" ::: "memory");
   // this warp's first group: its absmax values are in flight while the mean is formed
-  int64_t g = (int64_t)blockIdx.x * 8 + warp;
+  int64_t g = (int64_t)blockIdx.x * kDqWarps + warp;
   float a[8];
   auto load_group = [&](int64_t gg) {
     const int64_t b0 = gg * kB2 + lane * 8;
@@ -316,9 +413,9 @@ __global__ void __launch_bounds__(256) dq_mean_groups_kernel(const float* __rest
     }
   };
   if (g < ng) load_group(g);
-  const int64_t nchunks = (ng + 2047) / 2048;
+  const int64_t nchunks = (ng + kDqChunk - 1) / kDqChunk;
   for (int64_t ch = 0; ch < nchunks; ++ch) {
-    const int64_t i0 = ch * 2048 + 8 * (int64_t)threadIdx.x;
+    const int64_t i0 = ch * kDqChunk + 8 * (int64_t)threadIdx.x;
     double x[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) x[i] = (i0 + i < ng) ? gsum[i0 + i] : 0.0;
@@ -327,9 +424,13 @@ __global__ void __launch_bounds__(256) dq_mean_groups_kernel(const float* __rest
     for (int off = 1; off < 32; off <<= 1) s = s + __shfl_xor_sync(0xFFFFFFFFu, s, off);
     if (lane == 0) warp_sum[warp] = s;
     __syncthreads();
-    if (threadIdx.x == 0)
-      chunk_sum[ch] = ((warp_sum[0] + warp_sum[1]) + (warp_sum[2] + warp_sum[3])) +
-                      ((warp_sum[4] + warp_sum[5]) + (warp_sum[6] + warp_sum[7]));
+    if (warp == 0) {
+      // the 32 warp sums, in order, by the same butterfly
+      double w = warp_sum[lane];
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) w = w + __shfl_xor_sync(0xFFFFFFFFu, w, off);
+      if (lane == 0) chunk_sum[ch] = w;
+    }
     __syncthreads();
   }
   float mean;
@@ -356,7 +457,7 @@ __global__ void __launch_bounds__(256) dq_mean_groups_kernel(const float* __rest
     mean = __double2float_rn(warp_sum[0] / (double)nb);
   }
   if (blockIdx.x == 0 && threadIdx.x == 0) mean_out[0] = mean;
-  for (; g < ng; g += (int64_t)gridDim.x * 8) {
+  for (; g < ng; g += (int64_t)gridDim.x * kDqWarps) {
     float d[8];
     float m = 0.0f;
 #pragma unroll
@@ -365,7 +466,7 @@ __global__ void __launch_bounds__(256) dq_mean_groups_kernel(const float* __rest
       d[i] = (b < nb) ? __fsub_rn(a[i], mean) : 0.0f;
       m = fmaxf(m, fabsf(d[i]));
     }
-    if (g + (int64_t)gridDim.x * 8 < ng) load_group(g + (int64_t)gridDim.x * 8);
+    if (g + (int64_t)gridDim.x * kDqWarps < ng) load_group(g + (int64_t)gridDim.x * kDqWarps);
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
     uint32_t e[8];
@@ -485,7 +586,7 @@ cudaError_t launch_quantize(const CUtensorMap* w_map, const uint16_t* W, int64_t
                             double* gsum_ws, cudaStream_t st, int sw_encode) {
   const int64_t nb = (numel + kB1 - 1) / kB1;
   const int64_t ng = (nb + kB2 - 1) / kB2;
-  if (ng > (int64_t)kMaxMeanChunks * 2048) return cudaErrorInvalidValue;
+  if (ng > (int64_t)kMaxMeanChunks * kDqChunk) return cudaErrorInvalidValue;
   int sms = 148;
   int dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -511,8 +612,8 @@ cudaError_t launch_quantize(const CUtensorMap* w_map, const uint16_t* W, int64_t
   // The double-quantization kernel may launch while the quantize grid drains (programmatic
   // dependent launch); it waits for that grid's results before reading them.
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)grid_for((ng + 7) / 8, 1, 2 * sms));
-  cfg.blockDim = dim3(256);
+  cfg.gridDim = dim3((unsigned)grid_for((ng + kDqWarps - 1) / kDqWarps, 1, sms));
+  cfg.blockDim = dim3(kDqThreads);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];

@@ -19,6 +19,7 @@ enum : uint32_t {
   kErrWaitProducer = 1u << 1,  // a wait for the dequant producer ran out
   kErrWaitMma = 1u << 2,       // a wait for MMA completion ran out
   kErrWaitEmpty = 1u << 3,     // a wait for a free pipeline stage ran out
+  kErrWaitGroup = 1u << 4,     // a wait for the other warps of a quantize group ran out
 };
 
 // Bit flags raised by kernels whose bounded waits ran out (one word per device).  The
