@@ -10,9 +10,11 @@
 //
 // The tensor cores multiply exact bf16 values (x, dY, A, B, or an exact three-term bf16
 // split of an fp32 t or u: fp32 = t1 + t2 + t3 with 8 significant bits each) and accumulate
-// one 64-wide k-block at a time in TMEM (fp32).  After every k-block eight flush warps move
+// one 64-wide k-block at a time in TMEM (fp32); the three split terms of a k-block go into the
+// same accumulator (their products are exact, so the block sum carries fp32 accumulation
+// rounding only, as three separate sums would).  After every k-block eight flush warps move
 // the block sums into float64 registers (up to four TMEM accumulator buffers, so the next
-// k-blocks' MMAs overlap the flush), adding the three split terms of a column in float64.  The float64
+// k-blocks' MMAs overlap the flush).  The float64
 // partial of each K split goes to the workspace; a finalize kernel sums the splits.  With
 // the long reductions here (thousands of tokens), plain fp32 accumulation leaves errors far
 // above the elementwise absolute floor at outputs that cancel to near zero; this keeps the
@@ -42,7 +44,7 @@ constexpr bool kLrSpin = true;
 
 template <int BJ, int TERMS>
 struct LrCfg {
-  static constexpr int BN = BJ * TERMS;            // UMMA N
+  static constexpr int BN = BJ;                    // UMMA N (the split terms share the accumulator)
   static constexpr int kABytes = 128 * 64 * 2;
   static constexpr int kBTermBytes = BJ * 64 * 2;
   static constexpr int kBBytes = TERMS * kBTermBytes;
@@ -68,18 +70,22 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16_lr(uint32_t taddr, uint32_t (
       : "r"(taddr));
 }
 
-// One 64-deep k-block into a fresh accumulator: four unrolled 16-deep MMAs whose
-// descriptors differ only in the start address field.
-template <int BN, bool A_MN>
-__device__ __forceinline__ void lr_kblock(uint32_t d, uint32_t a_addr, uint32_t b_addr) {
+// One 64-deep k-block into a fresh accumulator: for each B term (the k-block's A tile times
+// that term's tile), four unrolled 16-deep MMAs whose descriptors differ only in the start
+// address field.
+template <int BN, int TERMS, bool A_MN>
+__device__ __forceinline__ void lr_kblock(uint32_t d, uint32_t a_addr, uint32_t b_addr, uint32_t b_term_bytes) {
   constexpr uint32_t idesc = umma_idesc_bf16(128, BN, A_MN ? 1u : 0u, 0u);
   const uint64_t a0 = A_MN ? umma_sdesc_sw128(a_addr, 8192u, 1024u) : umma_sdesc_sw128(a_addr, 16u, 1024u);
-  const uint64_t b0 = umma_sdesc_sw128(b_addr, 16u, 1024u);
 #pragma unroll
-  for (int k16 = 0; k16 < 4; ++k16) {
-    const uint64_t ad = a0 + (uint64_t)((A_MN ? 2048u : 32u) * (uint32_t)k16 >> 4);
-    const uint64_t bd = b0 + (uint64_t)(32u * (uint32_t)k16 >> 4);
-    umma_bf16(d, ad, bd, idesc, k16 > 0 ? 1u : 0u);
+  for (int t = 0; t < TERMS; ++t) {
+    const uint64_t b0 = umma_sdesc_sw128(b_addr + (uint32_t)t * b_term_bytes, 16u, 1024u);
+#pragma unroll
+    for (int k16 = 0; k16 < 4; ++k16) {
+      const uint64_t ad = a0 + (uint64_t)((A_MN ? 2048u : 32u) * (uint32_t)k16 >> 4);
+      const uint64_t bd = b0 + (uint64_t)(32u * (uint32_t)k16 >> 4);
+      umma_bf16(d, ad, bd, idesc, (t > 0 || k16 > 0) ? 1u : 0u);
+    }
   }
 }
 
@@ -191,16 +197,18 @@ __global__ void __launch_bounds__(kLrThreads, 1) lowrank_kernel(const __grid_con
         const uint32_t b_addr = a_addr + C::kABytes;
         const uint32_t d = tmem_base + (uint32_t)(buf * C::BN);
         if (kb_begin + it != p.kblocks - 1 || p.k16_last == 4) {
-          if (p.a_mn) lr_kblock<C::BN, true>(d, a_addr, b_addr);
-          else lr_kblock<C::BN, false>(d, a_addr, b_addr);
+          if (p.a_mn) lr_kblock<C::BN, TERMS, true>(d, a_addr, b_addr, C::kBTermBytes);
+          else lr_kblock<C::BN, TERMS, false>(d, a_addr, b_addr, C::kBTermBytes);
         } else {
           const uint32_t idesc = umma_idesc_bf16(128, C::BN, p.a_mn ? 1u : 0u, 0u);
-          for (int k16 = 0; k16 < p.k16_last; ++k16) {
-            const uint64_t ad = p.a_mn ? umma_sdesc_sw128(a_addr + (uint32_t)k16 * 2048u, 8192u, 1024u)
-                                       : umma_sdesc_sw128(a_addr + (uint32_t)k16 * 32u, 16u, 1024u);
-            const uint64_t bd = umma_sdesc_sw128(b_addr + (uint32_t)k16 * 32u, 16u, 1024u);
-            umma_bf16(d, ad, bd, idesc, k16 > 0 ? 1u : 0u);
-          }
+          for (int t = 0; t < TERMS; ++t)
+            for (int k16 = 0; k16 < p.k16_last; ++k16) {
+              const uint64_t ad = p.a_mn ? umma_sdesc_sw128(a_addr + (uint32_t)k16 * 2048u, 8192u, 1024u)
+                                         : umma_sdesc_sw128(a_addr + (uint32_t)k16 * 32u, 16u, 1024u);
+              const uint64_t bd =
+                  umma_sdesc_sw128(b_addr + (uint32_t)t * C::kBTermBytes + (uint32_t)k16 * 32u, 16u, 1024u);
+              umma_bf16(d, ad, bd, idesc, (t > 0 || k16 > 0) ? 1u : 0u);
+            }
         }
         umma_commit(&empty[s]);
         umma_commit(&accfull[buf]);
@@ -230,17 +238,11 @@ __global__ void __launch_bounds__(kLrThreads, 1) lowrank_kernel(const __grid_con
         const uint32_t tb = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * C::BN + c0);
 #pragma unroll
         for (int j0 = 0; j0 < HALF; j0 += 16) {
-          uint32_t r[TERMS][16];
-#pragma unroll
-          for (int t = 0; t < TERMS; ++t) tmem_ld_32x32b_x16_lr(tb + (uint32_t)(t * BJ + j0), r[t]);
+          uint32_t r[16];
+          tmem_ld_32x32b_x16_lr(tb + (uint32_t)j0, r);
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            double v = (double)__uint_as_float(r[0][j]);
-#pragma unroll
-            for (int t = 1; t < TERMS; ++t) v += (double)__uint_as_float(r[t][j]);
-            acc[j0 + j] += v;
-          }
+          for (int j = 0; j < 16; ++j) acc[j0 + j] += (double)__uint_as_float(r[j]);
         }
       }
       tc_fence_before();
