@@ -320,13 +320,6 @@ __device__ __forceinline__ uint64_t l2_policy_evict_last() {
   asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
   return pol;
 }
-// Streamed operands (activations: each k-slice is read by the CTAs of one column tile at about
-// the same time, then never again) leave L2 first, so that the codes stay resident.
-__device__ __forceinline__ uint64_t l2_policy_evict_first() {
-  uint64_t pol;
-  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
-  return pol;
-}
 // TMA tile load with an L2 cache-eviction hint (no multicast).
 __device__ __forceinline__ void tma_load_2d_hint(void* smem_dst, const CUtensorMap* map, int32_t x, int32_t y,
                                                  uint64_t* bar, uint64_t policy) {
@@ -452,7 +445,6 @@ __global__ void __launch_bounds__(Cfg<BN, A_TMEM>::kThreads, 1) qlora_gemm_kerne
     // ------------------------------------------------------------------ TMA producers
     const int tw = (warp == 0) ? 0 : 1;
     const uint64_t codes_policy = l2_policy_evict_last();   // the codes are re-read by every column tile
-    const uint64_t act_policy = l2_policy_evict_first();     // activations stream through
     int last_issue[8];            // phase of the last load issued into each stage (-1: none)
     for (int s = 0; s < 8; ++s) last_issue[s] = -1;
     bool ok = true;
@@ -482,11 +474,11 @@ __global__ void __launch_bounds__(Cfg<BN, A_TMEM>::kThreads, 1) qlora_gemm_kerne
       const int row0 = ki.ti.row0, col0 = ki.ti.col0;
       const int k = sg.a_k0 + ip.kb * kBK;
       int map = -1, cx = 0, cy = 0;
-      bool codes = false, act = false;
+      bool codes = false;
       uint8_t* dst = nullptr;
       uint64_t* bar = &full[s];
       if (lane == 0) {
-        map = sg.b_map; dst = stage_b(s); cx = sg.b_k0 + ip.kb * kBK; cy = col0; act = nf4;
+        map = sg.b_map; dst = stage_b(s); cx = sg.b_k0 + ip.kb * kBK; cy = col0;
       } else if (lane == 1) {
         if (sg.a_src == kANf4K) {
           if (!GENERIC) { map = sg.a_map; dst = stage_c(s); cx = k / 2; cy = row0; bar = A_TMEM ? &full[s] : &cfull[s]; codes = true; }
@@ -501,7 +493,7 @@ __global__ void __launch_bounds__(Cfg<BN, A_TMEM>::kThreads, 1) qlora_gemm_kerne
         map = sg.a_map; dst = stage_a(s) + 8192; cx = row0 + 64; cy = k;
       }
       if (map >= 0) {
-        if (codes || act) tma_load_2d_hint(dst, &p.maps[map], cx, cy, bar, codes ? codes_policy : act_policy);
+        if (codes) tma_load_2d_hint(dst, &p.maps[map], cx, cy, bar, codes_policy);
         else tma_load_2d(dst, &p.maps[map], cx, cy, bar);
       }
       __syncwarp();
