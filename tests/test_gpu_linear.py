@@ -136,3 +136,13 @@ def test_token_counts_cover_every_tile_width(M):
         W = synth.normal_bf16((N, K), 0.02, seed)
         inp = synth.linear_inputs(M, N, K, 32, seed + 100)
         _check(W, inp["x"], inp["A"], inp["B"], inp["dY"], 0.5, tag=f"M={M} N={N} K={K}")
+
+
+@pytest.mark.parametrize("M", [256, 300])
+def test_dx_256_token_tiles_on_ragged_edges(M):
+    """256-token tiles of the fused dX with K % 128 = 64 (the last row tile's second half lies
+    past the weight) and N % 64 != 0 (the last k-block of W rows is partial)."""
+    N, K = 200, 192
+    W = synth.normal_bf16((N, K), 0.02, 61)
+    inp = synth.linear_inputs(M, N, K, 64, 62)
+    _check(W, inp["x"], inp["A"], inp["B"], inp["dY"], 0.25, tag=f"ragged dX M={M}")
