@@ -10,12 +10,16 @@
 //
 // The tensor cores multiply exact bf16 values (x, dY, A, B, or an exact three-term bf16
 // split of an fp32 t or u: fp32 = t1 + t2 + t3 with 8 significant bits each) and accumulate
-// one 64-wide k-block at a time in TMEM (fp32); the three split terms of a k-block go into the
-// same accumulator (their products are exact, so the block sum carries fp32 accumulation
-// rounding only, as three separate sums would).  After every k-block eight flush warps move
-// the block sums into float64 registers (up to four TMEM accumulator buffers, so the next
-// k-blocks' MMAs overlap the flush).  The float64
-// partial of each K split goes to the workspace; a finalize kernel sums the splits.  With
+// one 64-wide k-block at a time in TMEM (fp32), one column group per split term.  After every
+// k-block eight flush warps add the block sums into a running sum held as an unevaluated pair
+// of fp32 values (hi + lo, about 48 significant bits: each block sum enters hi by an exact
+// two-sum and the rounding error goes to lo), with up to four TMEM accumulator buffers so
+// that the next k-blocks' MMAs overlap the flush.  The three split terms' block sums of a
+// column are first added in fp32, smallest first: one more rounding of the block sum's size,
+// the same order as the block's own fp32 accumulation.  (A float64 running sum did the same,
+// but the fp32 -> fp64 conversions run on a quarter-rate unit and paced the kernel.)  The
+// partial (hi + lo in float64) of each K split goes to the workspace; a finalize kernel sums
+// the splits.  With
 // the long reductions here (thousands of tokens), plain fp32 accumulation leaves errors far
 // above the elementwise absolute floor at outputs that cancel to near zero; this keeps the
 // error at the level of one fp32 rounding per 64-wide block.
@@ -44,7 +48,7 @@ constexpr bool kLrSpin = true;
 
 template <int BJ, int TERMS>
 struct LrCfg {
-  static constexpr int BN = BJ;                    // UMMA N (the split terms share the accumulator)
+  static constexpr int BN = BJ * TERMS;            // UMMA N
   static constexpr int kABytes = 128 * 64 * 2;
   static constexpr int kBTermBytes = BJ * 64 * 2;
   static constexpr int kBBytes = TERMS * kBTermBytes;
@@ -70,23 +74,47 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16_lr(uint32_t taddr, uint32_t (
       : "r"(taddr));
 }
 
-// One 64-deep k-block into a fresh accumulator: for each B term (the k-block's A tile times
-// that term's tile), four unrolled 16-deep MMAs whose descriptors differ only in the start
-// address field.
-template <int BN, int TERMS, bool A_MN>
-__device__ __forceinline__ void lr_kblock(uint32_t d, uint32_t a_addr, uint32_t b_addr, uint32_t b_term_bytes) {
+// One 64-deep k-block into a fresh accumulator: four unrolled 16-deep MMAs whose
+// descriptors differ only in the start address field.
+template <int BN, bool A_MN>
+__device__ __forceinline__ void lr_kblock(uint32_t d, uint32_t a_addr, uint32_t b_addr) {
   constexpr uint32_t idesc = umma_idesc_bf16(128, BN, A_MN ? 1u : 0u, 0u);
   const uint64_t a0 = A_MN ? umma_sdesc_sw128(a_addr, 8192u, 1024u) : umma_sdesc_sw128(a_addr, 16u, 1024u);
+  const uint64_t b0 = umma_sdesc_sw128(b_addr, 16u, 1024u);
 #pragma unroll
-  for (int t = 0; t < TERMS; ++t) {
-    const uint64_t b0 = umma_sdesc_sw128(b_addr + (uint32_t)t * b_term_bytes, 16u, 1024u);
-#pragma unroll
-    for (int k16 = 0; k16 < 4; ++k16) {
-      const uint64_t ad = a0 + (uint64_t)((A_MN ? 2048u : 32u) * (uint32_t)k16 >> 4);
-      const uint64_t bd = b0 + (uint64_t)(32u * (uint32_t)k16 >> 4);
-      umma_bf16(d, ad, bd, idesc, (t > 0 || k16 > 0) ? 1u : 0u);
-    }
+  for (int k16 = 0; k16 < 4; ++k16) {
+    const uint64_t ad = a0 + (uint64_t)((A_MN ? 2048u : 32u) * (uint32_t)k16 >> 4);
+    const uint64_t bd = b0 + (uint64_t)(32u * (uint32_t)k16 >> 4);
+    umma_bf16(d, ad, bd, idesc, k16 > 0 ? 1u : 0u);
   }
+}
+
+// Two fp32 lanes as one register pair, for the sm_100 paired fp32 instructions (each lane is
+// rounded to nearest exactly as the scalar instruction would round it).
+__device__ __forceinline__ uint64_t pair_of(uint32_t lo_bits, uint32_t hi_bits) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo_bits), "r"(hi_bits));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+// (hi, lo) += v for both lanes: s = hi + v and its exact error e (the two-sum: e = (hi - (s -
+// b)) + (v - b) with b = s - hi, exact in round-to-nearest without overflow), then hi = s and
+// lo = lo + e.  hi + lo carries about 48 significant bits over the whole reduction.
+__device__ __forceinline__ void two_sum_acc(uint64_t& hi, uint64_t& lo, uint64_t v) {
+  const uint64_t s = f2_add(hi, v);
+  const uint64_t b = f2_sub(s, hi);
+  const uint64_t e = f2_add(f2_sub(hi, f2_sub(s, b)), f2_sub(v, b));
+  hi = s;
+  lo = f2_add(lo, e);
 }
 
 template <int BJ, int TERMS>
@@ -197,18 +225,16 @@ __global__ void __launch_bounds__(kLrThreads, 1) lowrank_kernel(const __grid_con
         const uint32_t b_addr = a_addr + C::kABytes;
         const uint32_t d = tmem_base + (uint32_t)(buf * C::BN);
         if (kb_begin + it != p.kblocks - 1 || p.k16_last == 4) {
-          if (p.a_mn) lr_kblock<C::BN, TERMS, true>(d, a_addr, b_addr, C::kBTermBytes);
-          else lr_kblock<C::BN, TERMS, false>(d, a_addr, b_addr, C::kBTermBytes);
+          if (p.a_mn) lr_kblock<C::BN, true>(d, a_addr, b_addr);
+          else lr_kblock<C::BN, false>(d, a_addr, b_addr);
         } else {
           const uint32_t idesc = umma_idesc_bf16(128, C::BN, p.a_mn ? 1u : 0u, 0u);
-          for (int t = 0; t < TERMS; ++t)
-            for (int k16 = 0; k16 < p.k16_last; ++k16) {
-              const uint64_t ad = p.a_mn ? umma_sdesc_sw128(a_addr + (uint32_t)k16 * 2048u, 8192u, 1024u)
-                                         : umma_sdesc_sw128(a_addr + (uint32_t)k16 * 32u, 16u, 1024u);
-              const uint64_t bd =
-                  umma_sdesc_sw128(b_addr + (uint32_t)t * C::kBTermBytes + (uint32_t)k16 * 32u, 16u, 1024u);
-              umma_bf16(d, ad, bd, idesc, (t > 0 || k16 > 0) ? 1u : 0u);
-            }
+          for (int k16 = 0; k16 < p.k16_last; ++k16) {
+            const uint64_t ad = p.a_mn ? umma_sdesc_sw128(a_addr + (uint32_t)k16 * 2048u, 8192u, 1024u)
+                                       : umma_sdesc_sw128(a_addr + (uint32_t)k16 * 32u, 16u, 1024u);
+            const uint64_t bd = umma_sdesc_sw128(b_addr + (uint32_t)k16 * 32u, 16u, 1024u);
+            umma_bf16(d, ad, bd, idesc, k16 > 0 ? 1u : 0u);
+          }
         }
         umma_commit(&empty[s]);
         umma_commit(&accfull[buf]);
@@ -225,9 +251,10 @@ __global__ void __launch_bounds__(kLrThreads, 1) lowrank_kernel(const __grid_con
     const bool active = c0 < BJ;
     const int q = warp & 3;
     const int row = row0 + 32 * q + lane;
-    double acc[HALF];
+    // running sums of columns (2i, 2i + 1) as paired fp32 hi and lo parts
+    uint64_t hi[HALF / 2], lo[HALF / 2];
 #pragma unroll
-    for (int j = 0; j < HALF; ++j) acc[j] = 0.0;
+    for (int j = 0; j < HALF / 2; ++j) hi[j] = lo[j] = 0ull;
     bool ok = true;
     for (int it = 0; it < n_iters; ++it) {
       const int buf = it % NB;
@@ -238,11 +265,16 @@ __global__ void __launch_bounds__(kLrThreads, 1) lowrank_kernel(const __grid_con
         const uint32_t tb = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * C::BN + c0);
 #pragma unroll
         for (int j0 = 0; j0 < HALF; j0 += 16) {
-          uint32_t r[16];
-          tmem_ld_32x32b_x16_lr(tb + (uint32_t)j0, r);
+          uint32_t r[TERMS][16];
+#pragma unroll
+          for (int t = 0; t < TERMS; ++t) tmem_ld_32x32b_x16_lr(tb + (uint32_t)(t * BJ + j0), r[t]);
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) acc[j0 + j] += (double)__uint_as_float(r[j]);
+          for (int j = 0; j < 16; j += 2) {
+            uint64_t v = pair_of(r[0][j], r[0][j + 1]);
+            if constexpr (TERMS == 3) v = f2_add(v, f2_add(pair_of(r[2][j], r[2][j + 1]), pair_of(r[1][j], r[1][j + 1])));
+            two_sum_acc(hi[(j0 + j) / 2], lo[(j0 + j) / 2], v);
+          }
         }
       }
       tc_fence_before();
@@ -254,7 +286,10 @@ __global__ void __launch_bounds__(kLrThreads, 1) lowrank_kernel(const __grid_con
 #pragma unroll
       for (int j = 0; j < HALF; ++j) {
         const int col = col0 + c0 + j;
-        if (col < p.cols) out[(int64_t)col * p.rows + row] = acc[j];
+        const uint64_t h = hi[j / 2], l = lo[j / 2];
+        const float hj = __uint_as_float((uint32_t)(j & 1 ? h >> 32 : h));
+        const float lj = __uint_as_float((uint32_t)(j & 1 ? l >> 32 : l));
+        if (col < p.cols) out[(int64_t)col * p.rows + row] = (double)hj + (double)lj;
       }
     }
     tc_fence_before();
