@@ -735,13 +735,16 @@ def rows_variants(dev, peaks, peak):
     sizes = [R * l.K + l.N * R for l in lins]
     params = [torch.zeros(n, dtype=torch.float32, device=dev) for n in sizes]
     grads = [torch.zeros(n, dtype=torch.bfloat16, device=dev) for n in sizes]
-    opt = q.PagedAdamW(params, None, lr=1e-4, paged=True)
-    ta = _time_calls(lambda: opt.step(grads), 10)
     nparam = sum(sizes)
-    opt.close()
-    adam = {"params": nparam, "ms": ta, "gbs": nparam * 22 / (ta * 1e6),
-            "note": "paged AdamW step over the 13B block's adapters (states in managed memory, paged in each step);"
-                    " 22 B per parameter (fp32 p, m, v read and written, bf16 g read)"}
+    adam = {"params": nparam, "bytes_per_param": 26,
+            "note": "AdamW step over the 13B block's adapters (7 tensors, one launch each); 26 B per parameter "
+                    "(fp32 p, m, v read and written, bf16 g read); 'device': states in plain device memory, "
+                    "'paged': states in managed memory, prefetched to the device before every step"}
+    for mode in ("device", "paged"):
+        opt = q.PagedAdamW(params, None, lr=1e-4, paged=(mode == "paged"))
+        ta = _time_calls(lambda: opt.step(grads), 10)
+        opt.close()
+        adam[mode] = {"ms": ta, "gbs": nparam * 26 / (ta * 1e6), "frac_hbm": nparam * 26 / (ta * 1e6) / peaks["hbm_gbs"]}
     return {"variants_13b_q": points, "merge_13b_q": merge, "adamw_13b_block": adam}
 
 
