@@ -95,16 +95,16 @@ def pick_bf16_peak(peaks: dict, clocks: dict):
 # ------------------------------------------------------------------------------------------
 # DRAM traffic of the fused GEMMs
 # ------------------------------------------------------------------------------------------
-# Bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum), averaged over the 7 launches
-# of a timed step, from one single-pass capture of this script's own run:
+# Bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum), averaged over the 14 launches
+# of the two timed steps, from one single-pass capture of this script's own run:
 #   ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum
-#       --clock-control none -k regex:qlora_gemm_kernel -c 42
-#       python bench.py --steps 2 --warmup 1 --no-e2e --no-cpu-baseline
+#       --clock-control none -k regex:"qlora_gemm|nf4_quant_stream|dq_mean|nf4_dequant|lowrank" -c 189
+#       python bench.py --steps 2 --warmup 1 --no-e2e --no-cpu-baseline --no-extra
 # They hold only for the kernel sources they were taken on: once any of FUSED_SOURCES changes
 # the traffic is reported as null.
 FUSED_SOURCES = ("gemm.cuh", "gemm.h", "common.cuh", "nf4_device.cuh", "qlora_nf4.cu")
-FUSED_TRAFFIC = {"sources_sha256": "3f9bcb1cf5cee1fd707ca405e578ba2ffa2eb7a0358265ff7aac3631c75b2d7b",
-                 "fwd": 272967095, "dx": 318708663}
+FUSED_TRAFFIC = {"sources_sha256": "3326052bb9d46653d75b10fbedb111935e2d7fa1632788b01d00fa305cf3dd17",
+                 "fwd": 280698642, "dx": 308967753}
 
 
 def fused_traffic(which: str):
