@@ -51,6 +51,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # Algorithmic bytes per weight: quantize reads bf16 (2 B) and writes codes (0.5 B), scale
 # codes (1/64 B) and group constants (4/(64*256) B); dequant reads the latter and writes bf16.
 CODEC_BYTES_PER_WEIGHT = 2.0 + 0.5 + 1.0 / 64 + 4.0 / (64 * 256)
+# float64 fused multiply-add peak of one B200, derived from unit counts and clock: 148 SMs x 64
+# float64 FMA per cycle per SM (ncu's peak_sustained for sm__sass_thread_inst_executed_op_dfma)
+# x 2 flops x 1.965 GHz (clocks.max.sm).  No measured figure exists for it.
+FP64_PEAK_TFLOPS = 148 * 64 * 2 * 1.965e9 / 1e12
 # kernels one nf4_quantize_dq call launches
 QUANTIZE_LAUNCHES = 2
 
@@ -729,8 +733,11 @@ def rows_variants(dev, peaks, peak):
     Q = q.nf4_quantize_dq(W)
     Ab, Bb = A, B * 20
     tm = _time_calls(lambda: q.merge_requantize(Q, Ab, Bb, s), 5)
+    fp64 = numel * R * 2 / (tm * 1e9)
     merge = {"shape": "5120x5120 r=64 NF4+DQ", "ms": tm, "gweights_per_s": numel / (tm * 1e6),
-             "note": "W'' = bf16(W' + s B A), float64 rank-r sum, then re-quantized; float64-bound"}
+             "fp64_tflops": fp64, "bound": "alu", "fp64_peak_tflops": FP64_PEAK_TFLOPS,
+             "frac_fp64": fp64 / FP64_PEAK_TFLOPS,
+             "note": "W'' = bf16(W' + s B A): float64 rank-r sum (2 r flops per weight), then re-quantized"}
     lins = linears()
     sizes = [R * l.K + l.N * R for l in lins]
     params = [torch.zeros(n, dtype=torch.float32, device=dev) for n in sizes]

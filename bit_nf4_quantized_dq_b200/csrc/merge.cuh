@@ -60,20 +60,24 @@ __device__ __forceinline__ float base_weight(const MergeParams& p, int64_t n, in
   return __bfloat162float(__float2bfloat16_rn(w));
 }
 
-// One CTA per tile of 32 rows x 64 columns; thread t owns row t / 8 and the 8 columns
-// 8 (t % 8) .. + 7.  The rank dimension goes through shared memory in chunks of 32, converted
-// to float64 (exactly) on the way in.
-constexpr int kMergeRows = 32, kMergeCols = 64, kMergeJ = 32;
+// One CTA per tile of 128 rows x 64 columns; thread t owns the 8 columns 8 (t % 8) .. + 7 of
+// the four rows t / 8 + 32 i (i = 0..3), so that each pair of shared-memory loads of A feeds 32
+// float64 fused multiply-adds.  The rank dimension goes through shared memory in chunks of 16,
+// converted to float64 (exactly) on the way in.  Each accumulator still runs over j = 0 .. r-1
+// in order.
+constexpr int kMergeRows = 128, kMergeCols = 64, kMergeJ = 16, kMergeRowsPerThread = 4;
 
 __global__ void __launch_bounds__(256) merge_dense_kernel(const __grid_constant__ MergeParams p) {
-  __shared__ double As[kMergeJ][kMergeCols];    // 16 KB
-  __shared__ double Bs[kMergeRows][kMergeJ + 1];
+  __shared__ __align__(16) double As[kMergeJ][kMergeCols];    // 8 KB
+  __shared__ double Bs[kMergeRows][kMergeJ + 1];               // 17 KB
   const int t = threadIdx.x;
   const int64_t n0 = (int64_t)blockIdx.y * kMergeRows, k0 = (int64_t)blockIdx.x * kMergeCols;
   const int rr = t >> 3, cc = (t & 7) * 8;
-  double acc[8];
+  double acc[kMergeRowsPerThread][8];
 #pragma unroll
-  for (int c = 0; c < 8; ++c) acc[c] = 0.0;
+  for (int i = 0; i < kMergeRowsPerThread; ++i)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[i][c] = 0.0;
   for (int j0 = 0; j0 < p.r; j0 += kMergeJ) {
     const int jn = (p.r - j0) < kMergeJ ? (p.r - j0) : kMergeJ;
     __syncthreads();
@@ -91,27 +95,41 @@ __global__ void __launch_bounds__(256) merge_dense_kernel(const __grid_constant_
     }
     __syncthreads();
     for (int j = 0; j < jn; ++j) {
-      const double b = Bs[rr][j];
+      double a[8];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) acc[c] = __fma_rn(b, As[j][cc + c], acc[c]);   // b * a is exact
+      for (int c = 0; c < 8; c += 2) {
+        const double2 a2 = *reinterpret_cast<const double2*>(&As[j][cc + c]);
+        a[c] = a2.x;
+        a[c + 1] = a2.y;
+      }
+#pragma unroll
+      for (int i = 0; i < kMergeRowsPerThread; ++i) {
+        const double b = Bs[rr + 32 * i][j];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[i][c] = __fma_rn(b, a[c], acc[i][c]);   // b * a is exact
+      }
     }
   }
-  const int64_t n = n0 + rr;
-  if (n >= p.N || k0 + cc >= p.K) return;                 // K % 8 == 0: whole groups of 8 in or out
-  uint32_t packed[4];
+  if (k0 + cc >= p.K) return;                              // K % 8 == 0: whole groups of 8 in or out
 #pragma unroll
-  for (int c = 0; c < 8; c += 2) {
-    uint32_t h[2];
+  for (int i = 0; i < kMergeRowsPerThread; ++i) {
+    const int64_t n = n0 + rr + 32 * i;
+    if (n >= p.N) break;
+    uint32_t packed[4];
 #pragma unroll
-    for (int d = 0; d < 2; ++d) {
-      const int64_t k = k0 + cc + c + d;
-      const double tterm = __dmul_rn(p.s, acc[c + d]);
-      const double v = __dadd_rn((double)base_weight(p, n, k), tterm);
-      h[d] = bf16_rn_from_f64(v);
+    for (int c = 0; c < 8; c += 2) {
+      uint32_t h[2];
+#pragma unroll
+      for (int d = 0; d < 2; ++d) {
+        const int64_t k = k0 + cc + c + d;
+        const double tterm = __dmul_rn(p.s, acc[i][c + d]);
+        const double v = __dadd_rn((double)base_weight(p, n, k), tterm);
+        h[d] = bf16_rn_from_f64(v);
+      }
+      packed[c / 2] = h[0] | (h[1] << 16);
     }
-    packed[c / 2] = h[0] | (h[1] << 16);
+    *reinterpret_cast<uint4*>(p.out + n * p.K + k0 + cc) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
   }
-  *reinterpret_cast<uint4*>(p.out + n * p.K + k0 + cc) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
 }
 
 static cudaError_t launch_merge_dense(const MergeParams& p, cudaStream_t st) {
