@@ -686,10 +686,30 @@ def rows_robust(L, dev, peaks, peak):
             row["gbs"] = hb / (ms * 1e6)
             if M <= 16:
                 row["frac_hbm"] = row["gbs"] / peaks["hbm_gbs"]
+                # the same calls replayed from a CUDA graph: the host-side cost of the Python
+                # calls (larger than the kernels at these sizes) leaves the timed region
+                try:
+                    torch.cuda.synchronize()
+                    side = torch.cuda.Stream()
+                    side.wait_stream(torch.cuda.current_stream())
+                    with torch.cuda.stream(side):
+                        fb()
+                    torch.cuda.current_stream().wait_stream(side)
+                    g = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(g):
+                        fb()
+                    mg = _time_calls(g.replay, 50)
+                    row["ms_graph"] = mg
+                    row["gbs_graph"] = hb / (mg * 1e6)
+                    row["frac_hbm_graph"] = row["gbs_graph"] / peaks["hbm_gbs"]
+                    del g
+                except Exception as exc:   # capture is a measurement aid; report why it is missing
+                    row["graph_error"] = str(exc)[:120]
             out.append(row)
     q.check_device_error()
     return {"workload": "robust_4000x3000", "points": out,
-            "note": "fwd + bwd through the Python binding (allocating outputs); M <= 16 is HBM-bound"}
+            "note": "fwd + bwd through the Python binding (allocating outputs); M <= 16 is HBM-bound, and is "
+                    "also timed as CUDA-graph replays of the same calls (ms_graph)"}
 
 
 def rows_variants(dev, peaks, peak):
