@@ -346,10 +346,25 @@ __device__ __forceinline__ void split3(double v, uint16_t& a, uint16_t& b, uint1
   c = __bfloat16_as_ushort(__float2bfloat16_rn((float)r2));
 }
 
+// sum_z p[z * stride] for z = 0 .. splits-1, added in that order; the loads of up to eight
+// splits are issued before their sum, so the splits' memory latencies overlap.
+__device__ __forceinline__ double sum_splits(const double* __restrict__ p, int splits, int64_t stride) {
+  double v = 0.0;
+  for (int z0 = 0; z0 < splits; z0 += 8) {
+    double x[8];
+#pragma unroll
+    for (int z = 0; z < 8; ++z) x[z] = (z0 + z < splits) ? p[(int64_t)(z0 + z) * stride] : 0.0;
+#pragma unroll
+    for (int z = 0; z < 8; ++z)
+      if (z0 + z < splits) v += x[z];
+  }
+  return v;
+}
+
 // Token-side result (t or u): v = alpha * sum_z partial[z][j][m].  Optional outputs:
 // fp32 [M][r]; bf16 hi / lo [M][r] (two-term split, for the fused GEMMs' adapter k-blocks);
 // the three-term split transposed, T3[term][j][m] with row pitch ldT (for dA / dB).
-// One 32 x 32 tile (m0.., j0..) per block of 32 x 32 threads: the partials are read along m,
+// One 32 x 32 tile (m0.., j0..) per block of 32 x 8 threads: the partials are read along m,
 // the [M][r] outputs written along j through a shared-memory transpose.
 __global__ void finalize_tokens_kernel(const double* __restrict__ partial, int splits, int64_t M, int64_t r,
                                        double alpha, float* __restrict__ f32, uint16_t* __restrict__ hi,
@@ -360,7 +375,7 @@ __global__ void finalize_tokens_kernel(const double* __restrict__ partial, int s
     const int64_t j = j0 + i, m = m0 + threadIdx.x;
     double v = 0.0;
     if (m < M && j < r) {
-      for (int z = 0; z < splits; ++z) v += partial[((int64_t)z * r + j) * M + m];
+      v = sum_splits(partial + j * M + m, splits, r * M);
       v *= alpha;
       if (T3) {
         uint16_t a, b, c;
@@ -410,7 +425,7 @@ __global__ void split3_T_kernel(const float* __restrict__ t, int64_t M, int64_t 
 
 // Feature-side gradient: g[j][i] = bf16(sum_z partial[z][j][i]); transpose_out = 0 writes
 // out[j * n + i] (dA, [r][K]), 1 writes out[i * r + j] (dB, [N][r]).  One 32 x 32 tile
-// (i0.., j0..) per block of 32 x 32 threads; the transposed case goes through shared memory so
+// (i0.., j0..) per block of 32 x 8 threads; the transposed case goes through shared memory so
 // that both the partials and the output are accessed along their rows.
 __global__ void finalize_grad_kernel(const double* __restrict__ partial, int splits, int64_t r, int64_t n,
                                      uint16_t* __restrict__ out, int transpose_out) {
@@ -420,8 +435,7 @@ __global__ void finalize_grad_kernel(const double* __restrict__ partial, int spl
     const int64_t j = j0 + a, i = i0 + threadIdx.x;
     uint16_t g = 0;
     if (i < n && j < r) {
-      double v = 0.0;
-      for (int z = 0; z < splits; ++z) v += partial[((int64_t)z * r + j) * n + i];
+      const double v = sum_splits(partial + j * n + i, splits, r * n);
       g = bf16_bits_rn(v);
       if (!transpose_out) out[j * n + i] = g;
     }
@@ -439,7 +453,7 @@ static cudaError_t launch_finalize_tokens(const double* partial, int splits, int
                                           float* f32, uint16_t* hi, uint16_t* lo, uint16_t* T3, int64_t ldT,
                                           cudaStream_t st) {
   dim3 grid((unsigned)((M + 31) / 32), (unsigned)((r + 31) / 32));
-  finalize_tokens_kernel<<<grid, dim3(32, 32), 0, st>>>(partial, splits, M, r, alpha, f32, hi, lo, T3, ldT);
+  finalize_tokens_kernel<<<grid, dim3(32, 8), 0, st>>>(partial, splits, M, r, alpha, f32, hi, lo, T3, ldT);
   return cudaGetLastError();
 }
 
@@ -453,7 +467,7 @@ static cudaError_t launch_split3_T(const float* t, int64_t M, int64_t r, uint16_
 static cudaError_t launch_finalize_grad(const double* partial, int splits, int64_t r, int64_t n, uint16_t* out,
                                         int transpose_out, cudaStream_t st) {
   dim3 grid((unsigned)((n + 31) / 32), (unsigned)((r + 31) / 32));
-  finalize_grad_kernel<<<grid, dim3(32, 32), 0, st>>>(partial, splits, r, n, out, transpose_out);
+  finalize_grad_kernel<<<grid, dim3(32, 8), 0, st>>>(partial, splits, r, n, out, transpose_out);
   return cudaGetLastError();
 }
 
