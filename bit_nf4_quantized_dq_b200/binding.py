@@ -29,6 +29,7 @@ SIGNATURES = {
     "qnf4_version": (c_int, []),
     "qnf4_last_error": (ctypes.c_char_p, []),
     "qnf4_device_error": (c_int, [c_void_p, ctypes.POINTER(ctypes.c_uint32)]),
+    "qnf4_selftest_bounded_wait": (c_int, [ctypes.c_uint64, c_void_p]),
     "nf4_quantize_workspace_bytes": (c_size_t, [c_int64]),
     "nf4_quantize_dq": (c_int, [c_void_p, c_int64, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                 c_size_t, c_void_p]),

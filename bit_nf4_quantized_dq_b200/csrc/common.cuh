@@ -20,6 +20,7 @@ enum : uint32_t {
   kErrWaitMma = 1u << 2,       // a wait for MMA completion ran out
   kErrWaitEmpty = 1u << 3,     // a wait for a free pipeline stage ran out
   kErrWaitGroup = 1u << 4,     // a wait for the other warps of a quantize group ran out
+  kErrWaitSelfTest = 1u << 5,  // the bounded-wait self-test's wait ran out (expected)
 };
 
 // Bit flags raised by kernels whose bounded waits ran out (one word per device).  The
@@ -107,12 +108,12 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
   return ok != 0;
 }
 // Bounded wait by one thread: returns false (and raises `flag` in the device error word and in
-// the CTA-local abort word) if the phase did not complete within kWaitLimitNs of wall-clock
-// time, or if another role of the CTA has already aborted.
+// the CTA-local abort word) if the phase did not complete within `limit_ns` (kWaitLimitNs unless
+// given) of wall-clock time, or if another role of the CTA has already aborted.
 // SPIN polls without a suspend hint (for hand-offs on the critical path of every k-block).
 template <bool CLUSTER_ACQUIRE = false, bool SPIN = false>
 __device__ __forceinline__ bool mbar_wait_thread(uint64_t* bar, uint32_t parity, volatile uint32_t* abort_word,
-                                                 uint32_t flag) {
+                                                 uint32_t flag, uint64_t limit_ns = kWaitLimitNs) {
   auto poll = [&]() { return CLUSTER_ACQUIRE ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
   bool ok = poll();
   if (!ok) {
@@ -125,7 +126,7 @@ __device__ __forceinline__ bool mbar_wait_thread(uint64_t* bar, uint32_t parity,
       }
       if ((i & 15u) == 0u) {
         if (*abort_word) break;
-        if (global_timer_ns() - t0 > kWaitLimitNs) {
+        if (global_timer_ns() - t0 > limit_ns) {
           *abort_word = 1u;
           atomicOr(&g_error_word, flag);
           break;

@@ -441,6 +441,37 @@ int qnf4_device_error(void* stream, uint32_t* word) {
   return QNF4_OK;
 }
 
+namespace qnf4 {
+// The bounded-wait self-test: one thread waits on an mbarrier that nothing arrives at, through
+// the same helper every pipeline wait uses, so the wait must give up after `limit_ns`, raise its
+// flag in the device error word and return.
+__global__ void selftest_bounded_wait_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ uint32_t abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0u;
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    volatile uint32_t* abort_word = &abort_flag;
+    (void)mbar_wait_thread(&bar, 0u, abort_word, kErrWaitSelfTest, limit_ns);
+  }
+}
+}  // namespace qnf4
+
+int qnf4_selftest_bounded_wait(uint64_t limit_ns, void* stream) {
+  g_last_error.clear();
+  if (limit_ns < 1000000ull || limit_ns > 10000000000ull)
+    return fail(QNF4_ERR_INVALID, "limit_ns must lie in [1 ms, 10 s]");
+  if (int rc = check_arch()) return rc;
+  qnf4::selftest_bounded_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
+  return QNF4_OK;
+}
+
 size_t nf4_quantize_workspace_bytes(int64_t numel) { return qnf4_quantize_workspace_bytes_ex(numel, 1); }
 
 size_t qnf4_quantize_workspace_bytes_ex(int64_t numel, int double_quant) {

@@ -66,6 +66,14 @@ const char* qnf4_last_error(void);
  * pointer. */
 int qnf4_device_error(void* stream, uint32_t* word);
 
+/* Bounded-wait self-test (a diagnostic, no counterpart in the method): enqueues one kernel
+ * whose single waiting thread waits on a barrier that nothing completes, through the same
+ * bounded-wait code every pipeline wait of the library uses.  After `limit_ns` nanoseconds of
+ * wall-clock time (1 ms .. 10 s, else QNF4_ERR_INVALID) the wait gives up, sets bit 5 (0x20)
+ * of the device error word and the kernel returns; the CUDA context stays usable.  A following
+ * qnf4_device_error() returns QNF4_ERR_DEVICE with that bit set (and clears the word). */
+int qnf4_selftest_bounded_wait(uint64_t limit_ns, void* stream);
+
 /* ---------------------------------------------------------------------------------------
  * NF4 blockwise quantization with double quantization.
  * [T] section 3 (both levels), [E] steps 2-3.

@@ -65,6 +65,13 @@ def _fwd(L, M, K, N, r, ws_bytes=1 << 30, x=FAKE):
                               ws_bytes, None)
 
 
+def test_selftest_rejects_limits_outside_range_before_any_device_work():
+    L = binding.lib()
+    assert L.qnf4_selftest_bounded_wait(999_999, None) == -1          # below 1 ms
+    assert L.qnf4_selftest_bounded_wait(10_000_000_001, None) == -1   # above 10 s
+    assert b"limit_ns" in L.qnf4_last_error()
+
+
 def test_linear_shape_errors():
     L = binding.lib()
     assert _fwd(L, 128, 1024, 1024, 16, x=None) == -1
